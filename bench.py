@@ -1,0 +1,457 @@
+#!/usr/bin/env python
+"""Benchmark of the QLoRA NF4 linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload: the 7B attention projection, W 4096 x 4096 bf16 ~ N(0, 0.02^2)
+with 0.1 % outliers at +-8 sigma, NF4 blocksize 64 + double quantisation
+(256), LoRA r = 16, alpha = 32, X = 8 x 512 = 4096 tokens per GPU.  One step
+is the whole path over one batch: quantise W, forward, backward (dX, dA, dB).
+The metric counts the forward + backward FLOPs only (4MNK + 6Mr(N+K)), so the
+quantisation inside each step makes the number conservative.
+
+Three input sets (W, X, dY, outputs: ~170 MB each, 510 MB in all) rotate
+between steps so that no step finds its inputs in the 126 MB L2.
+
+With N > 1 (torchrun, one process per GPU) every rank holds the same frozen
+W and its own tokens; the LoRA gradients dA, dB are summed over ranks with
+one NCCL all-reduce per step (data parallelism; weak scaling).  Rank 0
+prints one JSON line.
+
+--impl reference times the CPU oracle (oracle/) on the host cores on a
+bounded sample of the same workload.
+"""
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+WORKLOAD = "attn_4096"
+TOKENS = 4096
+METRIC = "QLoRA linear fwd+bwd TFLOP/s and NF4 weight GB/s at 1 B200; % of roofline"
+UNIT = "TFLOP/s"
+N_SETS = 3
+
+
+def fwd_flops(M, N, K, r):
+    return 2 * M * N * K + 2 * M * K * r + 2 * M * N * r
+
+
+def fwd_bwd_flops(M, N, K, r):
+    return 4 * M * N * K + 6 * M * r * (N + K)
+
+
+def nf4_bytes(N, K, bs=64, dq=256):
+    n = N * K
+    nb = -(-n // bs)
+    return -(-n // 2) + nb + 4 * (-(-nb // dq)) + 4
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            d = json.load(fh)
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+def workload_config(n_gpus):
+    return {
+        "workload": "attn_4096: 7B attention projection, W 4096x4096 bf16 N(0,0.02^2) + 0.1% "
+                    "outliers at 8 sigma, NF4 b64 + double quant b256, LoRA r=16 alpha=32, "
+                    "M=4096 tokens (8x512) per GPU; step = quantise + fwd + bwd (dX, dA, dB)",
+        "global_batch": TOKENS * n_gpus,
+        "seq_len": 512,
+        "parallelism": f"dp{n_gpus}",
+        "l2": f"{N_SETS} rotating input sets (~510 MB) > 126 MB L2",
+    }
+
+
+# ------------------------------------------------------------------ clocks --
+
+class ClockSampler:
+    """nvidia-smi samples (200 ms) taken while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v == "Active"})
+        # samples under load: the upper half of the clock readings excludes idle gaps
+        return {"sm_mhz": statistics.median(c for c, _, _ in rows),
+                "sm_max_mhz": max(m for _, m, _ in rows), "samples": len(rows),
+                "reasons": reasons}
+
+
+# ----------------------------------------------------------- GPU arm -----
+
+class InputSet:
+    def __init__(self, shape, M, seed, rank, dev, Q, WL):
+        self.W = WL.weight(shape, seed, dev)
+        self.A = WL.lora_a(shape, seed, dev)
+        self.B = WL.lora_b(shape, seed, dev)
+        tok_seed = seed + 1000 * (rank + 1)
+        self.X = WL.activations(shape, M, tok_seed, dev)
+        self.dY = WL.grad_output(shape, M, tok_seed, dev)
+        N, K, r = shape.d_out, shape.d_in, shape.r
+        self.q = Q.QuantizedWeight.empty(N, K, 64, 256, Q.QLORA_TABLE_NF4, dev)
+        self.qws = torch.zeros(Q.qlora_nf4_sizes(N, K)["workspace"], dtype=torch.uint8, device=dev)
+        fwd_b, bwd_b = Q.qlora_linear_workspace(M, N, K, r)
+        self.fws = torch.zeros(fwd_b, dtype=torch.uint8, device=dev)
+        self.bws = torch.zeros(bwd_b, dtype=torch.uint8, device=dev)
+        self.Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        self.U = torch.empty((M, r), dtype=torch.float32, device=dev)
+        self.dX = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+        self.dA = torch.empty((r, K), dtype=torch.float32, device=dev)
+        self.dB = torch.empty((N, r), dtype=torch.float32, device=dev)
+
+
+def run_step(s, shape, Q, ev=None, world=1):
+    Q.qlora_quantize(s.W, out=s.q, workspace=s.qws, check=False)
+    if ev is not None:
+        ev[0].record()
+    Q.qlora_linear_fwd(s.q, s.A, s.B, shape.alpha, s.X, Y=s.Y, U_save=s.U, workspace=s.fws)
+    if ev is not None:
+        ev[1].record()
+    Q.qlora_linear_bwd(s.q, s.A, s.B, shape.alpha, s.X, s.U, s.dY, dX=s.dX, dA=s.dA, dB=s.dB,
+                       workspace=s.bws)
+    if ev is not None:
+        ev[2].record()
+    if world > 1:
+        torch.distributed.all_reduce(s.dA)
+        torch.distributed.all_reduce(s.dB)
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(value, world, dev):
+    if world == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def time_decode(Q, WL, dev, peaks, steps=30, warmup=5):
+    """Decode-shaped gate/up linear (11008 x 4096, r = 64) at M = 1 and 16:
+    forward + backward, 8 rotating weight copies (8 x 23 MB > L2)."""
+    shape = WL.WORKLOADS["mlp_11008"].linears[0]
+    N, K, r = shape.d_out, shape.d_in, shape.r
+    copies = []
+    for c in range(8):
+        W = WL.weight(shape, 7 * c, dev)
+        copies.append(Q.qlora_quantize(W))
+        del W
+    A, B = WL.lora_a(shape, 0, dev), WL.lora_b(shape, 0, dev)
+    out = {}
+    for M in (1, 16):
+        X, dY = WL.activations(shape, M, 3, dev), WL.grad_output(shape, M, 3, dev)
+        fb, bb = Q.qlora_linear_workspace(M, N, K, r)
+        fws = torch.zeros(fb, dtype=torch.uint8, device=dev)
+        bws = torch.zeros(bb, dtype=torch.uint8, device=dev)
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        U = torch.empty((M, r), dtype=torch.float32, device=dev)
+        dX = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+        dA = torch.empty((r, K), dtype=torch.float32, device=dev)
+        dB = torch.empty((N, r), dtype=torch.float32, device=dev)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        for i in range(warmup + steps):
+            q = copies[i % 8]
+            e = evs[i - warmup] if i >= warmup else None
+            if e:
+                e[0].record()
+            Q.qlora_linear_fwd(q, A, B, shape.alpha, X, Y=Y, U_save=U, workspace=fws)
+            if e:
+                e[1].record()
+            Q.qlora_linear_bwd(q, A, B, shape.alpha, X, U, dY, dX=dX, dA=dA, dB=dB, workspace=bws)
+            if e:
+                e[2].record()
+        torch.cuda.synchronize()
+        t_f = statistics.median(e[0].elapsed_time(e[1]) for e in evs) * 1e-3
+        t_b = statistics.median(e[1].elapsed_time(e[2]) for e in evs) * 1e-3
+        wb = nf4_bytes(N, K)
+        out[f"M{M}"] = {
+            "fwd_us": round(t_f * 1e6, 2), "bwd_us": round(t_b * 1e6, 2),
+            "fwd_nf4_gbs": round(wb / t_f / 1e9, 1), "bwd_nf4_gbs": round(wb / t_b / 1e9, 1),
+            "fwd_frac_hbm": round(wb / t_f / 1e9 / peaks["hbm"], 4),
+            "bwd_frac_hbm": round(wb / t_b / 1e9 / peaks["hbm"], 4),
+        }
+    out["workload"] = "mlp gate/up 11008x4096, r=64, alpha=16; NF4 bytes per pass " \
+                      f"{nf4_bytes(N, K)}; 8 rotating weight copies; median of {steps}"
+    return out
+
+
+def cpu_oracle_sample(shape, tokens_sample, repeats, WL):
+    """Oracle quantise of the full W + fwd/bwd on `tokens_sample` tokens."""
+    import oracle
+    from threadpoolctl import threadpool_info
+    inp = WL.linear_inputs(shape, tokens_sample, 0)
+    W = inp["W"].float().numpy()
+    f = lambda t: t.float().numpy()
+    A, B, X, dY = f(inp["A"]), f(inp["B"]), f(inp["X"]), f(inp["dY"])
+    times = []
+    for _ in range(repeats):
+        t0 = time.perf_counter()
+        qt = oracle.quantize(W, 64, 256)
+        w_hat = oracle.dequantize(qt).reshape(W.shape)
+        oracle.linear_fwd(w_hat, A, B, shape.alpha, X)
+        oracle.linear_bwd(w_hat, A, B, shape.alpha, X, dY)
+        times.append(time.perf_counter() - t0)
+    cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    t = statistics.median(times)
+    flops = fwd_bwd_flops(tokens_sample, shape.d_out, shape.d_in, shape.r)
+    return {"value": flops / t / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"oracle quantise of the full 4096x4096 W + fwd/bwd on {tokens_sample} of "
+                      f"the {TOKENS} tokens, median of {repeats}; FLOPs of those tokens / time",
+            "seconds_per_sample": round(t, 3)}
+
+
+def run_ours(args):
+    from bit_nf4_quantized_17_b200 import qlora as Q
+    from bit_nf4_quantized_17_b200 import workloads as WL
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+    peaks = measured_peaks()
+    shape = WL.WORKLOADS[WORKLOAD].linears[0]
+    N, K, r, M = shape.d_out, shape.d_in, shape.r, TOKENS
+    sets = [InputSet(shape, M, 100 * i, rank, dev, Q, WL) for i in range(N_SETS)]
+    torch.cuda.synchronize()
+
+    for i in range(args.warmup):
+        run_step(sets[i % N_SETS], shape, Q, world=world)
+    torch.cuda.synchronize()
+    barrier(world)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = Q.qlora_launch_count()
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        start.record()
+        for i in range(args.steps):
+            run_step(sets[i % N_SETS], shape, Q, ev=evs[i], world=world)
+        end.record()
+        torch.cuda.synchronize()
+        barrier(world)
+    launches = Q.qlora_launch_count() - launches0
+    elapsed_ms = max_over_ranks(start.elapsed_time(end), world, dev)
+    ms_per_step = elapsed_ms / args.steps
+    flops_step = fwd_bwd_flops(M, N, K, r)
+    value = flops_step * world / (ms_per_step * 1e-3) / 1e12
+    t_fwd = statistics.mean(e[0].elapsed_time(e[1]) for e in evs) * 1e-3
+    t_bwd = statistics.mean(e[1].elapsed_time(e[2]) for e in evs) * 1e-3
+
+    # roofline of the dominant kernel: the fused forward GEMM, timed as the
+    # whole forward call (its LoRA pre-GEMM included, so "achieved" is a lower bound)
+    achieved = fwd_flops(M, N, K, r) / t_fwd / 1e12
+    roofline = {"bound": "tensor", "achieved": round(achieved, 2),
+                "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
+                "frac": round(achieved / peaks["bf16_sustained"], 4),
+                "traffic": None,
+                "kernel": "forward call (LoRA pre-GEMM + fused dequant GEMM)",
+                "peak_kind": f"{peaks['source']} sustained bf16 (kernel timed inside a long step)"}
+
+    # end to end: host (pinned) inputs copied in, results copied out, every step
+    e2e = None
+    if not args.no_e2e:
+        s = sets[0]
+        host = {k: getattr(s, k).cpu().pin_memory() for k in ("W", "A", "B", "X", "dY")}
+        outs = {k: torch.empty_like(getattr(s, k), device="cpu").pin_memory()
+                for k in ("Y", "dX", "dA", "dB")}
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = sum(t.numel() * t.element_size() for t in outs.values())
+
+        def e2e_step():
+            for k, t in host.items():
+                getattr(s, k).copy_(t, non_blocking=True)
+            run_step(s, shape, Q, world=world)
+            for k, t in outs.items():
+                t.copy_(getattr(s, k), non_blocking=True)
+
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record()
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / args.steps
+        e2e = {"value": round(flops_step * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
+               "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h,
+               "path": "pinned host -> device copies, qlora_quantize + qlora_linear_fwd + "
+                       "qlora_linear_bwd through the C ABI, device -> pinned host copies"}
+
+    decode = None
+    if rank == 0 and world == 1 and not args.no_decode:
+        decode = time_decode(Q, WL, dev, peaks)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_oracle_sample(shape, 64, 3, WL)
+
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return
+    wb = nf4_bytes(N, K)
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,.) tensors of the workload's shapes)",
+        "config": workload_config(world),
+        "nf4_weight_gbs": round(2 * wb / (t_fwd + t_bwd) / 1e9, 1),
+        "fwd_ms": round(t_fwd * 1e3, 4), "bwd_ms": round(t_bwd * 1e3, 4),
+        "fwd_tflops": round(fwd_flops(M, N, K, r) / t_fwd / 1e12, 2),
+        "bwd_tflops": round((fwd_bwd_flops(M, N, K, r) - fwd_flops(M, N, K, r)) / t_bwd / 1e12, 2),
+        "frac_of_bf16_peak": round(value / world / peaks["bf16_sustained"], 4),
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": launches, "clocks": clk.summary(), "decode": decode,
+        "peaks": peaks,
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------ reference arm ----
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    from threadpoolctl import threadpool_info
+
+    import oracle
+    from bit_nf4_quantized_17_b200 import workloads as WL
+
+    shape = WL.WORKLOADS[WORKLOAD].linears[0]
+    ms = 32
+    inp = WL.linear_inputs(shape, ms, 0)
+    W = inp["W"].float().numpy()
+    f = lambda t: t.float().numpy()
+    A, B, X, dY = f(inp["A"]), f(inp["B"]), f(inp["X"]), f(inp["dY"])
+
+    def step():
+        qt = oracle.quantize(W, 64, 256)
+        w_hat = oracle.dequantize(qt).reshape(W.shape)
+        oracle.linear_fwd(w_hat, A, B, shape.alpha, X)
+        oracle.linear_bwd(w_hat, A, B, shape.alpha, X, dY)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    t = (time.perf_counter() - t0) / args.steps
+    flops = fwd_bwd_flops(ms, shape.d_out, shape.d_in, shape.r)
+    value = flops / t / 1e12
+    cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    sample = (f"oracle quantise of the full 4096x4096 W + fwd/bwd on {ms} of the {TOKENS} "
+              f"tokens per step; FLOPs of those tokens / time")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,.) tensors of the workload's shapes)",
+        "config": workload_config(world),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

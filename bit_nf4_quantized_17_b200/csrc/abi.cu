@@ -1,0 +1,212 @@
+// C ABI of libqlora.so: argument checks on the host, then kernel launches on
+// the caller's stream.  See include/qlora.h for the contract of each call.
+#include <atomic>
+#include <cstring>
+#include <mutex>
+
+#include "internal.cuh"
+#include "kernels.cuh"
+#include "linear.cuh"
+
+using namespace qlora;
+
+namespace {
+std::atomic<uint64_t> g_launches{0};
+}  // namespace
+
+void qlora::count_launch(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+namespace {
+
+constexpr int64_t kMaxElems = int64_t(1) << 36;
+
+bool pow2_in(int32_t v, int32_t lo, int32_t hi) {
+  return v >= lo && v <= hi && (v & (v - 1)) == 0;
+}
+
+const LevelTable* level_table(int32_t table) {
+  static LevelTable tabs[2];
+  static qlora_status ok[2];
+  static std::once_flag once;
+  std::call_once(once, [] {
+    ok[0] = make_level_table(QLORA_TABLE_NF4, &tabs[0]);
+    ok[1] = make_level_table(QLORA_TABLE_UNIFORM, &tabs[1]);
+  });
+  if (table < 0 || table > 1 || ok[table] != QLORA_OK) return nullptr;
+  return &tabs[table];
+}
+
+qlora_status check_nf4_shape(const qlora_nf4& q) {
+  if (q.rows < 1 || q.cols < 1 || q.rows > kMaxElems / q.cols) return QLORA_ERR_SHAPE;
+  if (!pow2_in(q.blocksize, 64, 1024)) return QLORA_ERR_UNSUPPORTED;
+  if (q.dq_blocksize != 0 && !pow2_in(q.dq_blocksize, 64, 1024)) return QLORA_ERR_UNSUPPORTED;
+  if (q.table != QLORA_TABLE_NF4 && q.table != QLORA_TABLE_UNIFORM) return QLORA_ERR_UNSUPPORTED;
+  return QLORA_OK;
+}
+
+qlora_status check_nf4_ptrs(const qlora_nf4& q) {
+  if (!q.codes || !q.factors) return QLORA_ERR_NULL;
+  if (q.dq_blocksize && (!q.scale_codes || !q.mean)) return QLORA_ERR_NULL;
+  if (!aligned16(q.codes) || !aligned16(q.factors)) return QLORA_ERR_ALIGN;
+  if (q.dq_blocksize && (!aligned16(q.scale_codes) || !aligned16(q.mean))) return QLORA_ERR_ALIGN;
+  return QLORA_OK;
+}
+
+size_t quantize_workspace(int64_t n, int32_t bs, int32_t dq) {
+  const int64_t nb = ceil_div(n, bs);
+  return dq ? 512 + static_cast<size_t>(ceil_div(4 * nb, 256) * 256) : 512;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* qlora_status_string(qlora_status s) {
+  switch (s) {
+    case QLORA_OK: return "ok";
+    case QLORA_ERR_NULL: return "a required pointer is NULL";
+    case QLORA_ERR_ALIGN: return "a device pointer is not 16-byte aligned";
+    case QLORA_ERR_SHAPE: return "a size is out of range or sizes disagree";
+    case QLORA_ERR_UNSUPPORTED: return "request not supported by this build";
+    case QLORA_ERR_NONFINITE: return "non-finite weight met while quantising";
+    case QLORA_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait gave up";
+    case QLORA_ERR_CUDA: return "a CUDA runtime call or kernel launch failed";
+    case QLORA_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+qlora_status qlora_levels(int32_t table, float levels_out[16]) {
+  if (!levels_out) return QLORA_ERR_NULL;
+  const LevelTable* t = level_table(table);
+  if (!t) return QLORA_ERR_UNSUPPORTED;
+  std::memcpy(levels_out, t->level, sizeof(float) * 16);
+  return QLORA_OK;
+}
+
+qlora_status qlora_nf4_sizes(int64_t rows, int64_t cols, int32_t blocksize, int32_t dq_blocksize,
+                             size_t* codes_bytes, size_t* scale_codes_bytes, size_t* factors_bytes,
+                             size_t* mean_bytes, size_t* workspace_bytes) {
+  qlora_nf4 q{};
+  q.rows = rows;
+  q.cols = cols;
+  q.blocksize = blocksize;
+  q.dq_blocksize = dq_blocksize;
+  qlora_status st = check_nf4_shape(q);
+  if (st != QLORA_OK) return st;
+  const int64_t n = rows * cols;
+  const int64_t nb = ceil_div(n, blocksize);
+  const int64_t ng = dq_blocksize ? ceil_div(nb, dq_blocksize) : 0;
+  if (codes_bytes) *codes_bytes = static_cast<size_t>(ceil_div(n, 2));
+  if (scale_codes_bytes) *scale_codes_bytes = dq_blocksize ? static_cast<size_t>(nb) : 0;
+  if (factors_bytes) *factors_bytes = static_cast<size_t>(4 * (dq_blocksize ? ng : nb));
+  if (mean_bytes) *mean_bytes = dq_blocksize ? 4 : 0;
+  if (workspace_bytes) *workspace_bytes = quantize_workspace(n, blocksize, dq_blocksize);
+  return QLORA_OK;
+}
+
+qlora_status qlora_quantize(const void* W, int32_t w_dtype, const qlora_nf4* q, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  if (!q || !W || !workspace) return QLORA_ERR_NULL;
+  qlora_status st = check_nf4_shape(*q);
+  if (st != QLORA_OK) return st;
+  if ((st = check_nf4_ptrs(*q)) != QLORA_OK) return st;
+  if (w_dtype != QLORA_F32 && w_dtype != QLORA_BF16) return QLORA_ERR_UNSUPPORTED;
+  if (!aligned16(W) || !aligned16(workspace)) return QLORA_ERR_ALIGN;
+  if (workspace_bytes < quantize_workspace(q->rows * q->cols, q->blocksize, q->dq_blocksize))
+    return QLORA_ERR_WORKSPACE;
+  const LevelTable* t = level_table(q->table);
+  if (!t) return QLORA_ERR_UNSUPPORTED;
+  return launch_quantize(W, w_dtype, *q, *t, workspace, static_cast<cudaStream_t>(stream));
+}
+
+qlora_status qlora_dequantize(const qlora_nf4* q, void* W_out, int32_t out_dtype, void* stream) {
+  if (!q || !W_out) return QLORA_ERR_NULL;
+  qlora_status st = check_nf4_shape(*q);
+  if (st != QLORA_OK) return st;
+  if ((st = check_nf4_ptrs(*q)) != QLORA_OK) return st;
+  if (out_dtype != QLORA_F32 && out_dtype != QLORA_BF16) return QLORA_ERR_UNSUPPORTED;
+  if (!aligned16(W_out)) return QLORA_ERR_ALIGN;
+  const LevelTable* t = level_table(q->table);
+  if (!t) return QLORA_ERR_UNSUPPORTED;
+  return launch_dequantize(*q, *t, W_out, out_dtype, static_cast<cudaStream_t>(stream));
+}
+
+qlora_status qlora_linear_workspace(int64_t M, int64_t N, int64_t K, int32_t r, size_t* fwd_bytes,
+                                    size_t* bwd_bytes) {
+  if (M < 0 || N < 1 || K < 1 || r < 1 || r > 256) return QLORA_ERR_SHAPE;
+  LinearPlan p = plan_linear(M, N, K, r);
+  if (fwd_bytes) *fwd_bytes = p.fwd_workspace;
+  if (bwd_bytes) *bwd_bytes = p.bwd_workspace;
+  return QLORA_OK;
+}
+
+static qlora_status check_linear(const qlora_nf4* W, const void* A, const void* B, int32_t r,
+                                 int64_t M, const void* X, const void* workspace,
+                                 size_t workspace_bytes, bool bwd) {
+  if (!W || !A || !B || !workspace || (M > 0 && !X)) return QLORA_ERR_NULL;
+  qlora_status st = check_nf4_shape(*W);
+  if (st != QLORA_OK) return st;
+  if ((st = check_nf4_ptrs(*W)) != QLORA_OK) return st;
+  if (W->blocksize != 64 || W->cols % 64 != 0) return QLORA_ERR_UNSUPPORTED;
+  if (r < 1 || r > 256 || M < 0) return QLORA_ERR_SHAPE;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(X) || !aligned16(workspace))
+    return QLORA_ERR_ALIGN;  // (a NULL X with M = 0 counts as aligned)
+  LinearPlan p = plan_linear(M, W->rows, W->cols, r);
+  if (workspace_bytes < (bwd ? p.bwd_workspace : p.fwd_workspace)) return QLORA_ERR_WORKSPACE;
+  if (!level_table(W->table)) return QLORA_ERR_UNSUPPORTED;
+  return QLORA_OK;
+}
+
+qlora_status qlora_linear_fwd(const qlora_nf4* W, const void* A, const void* B, int32_t r,
+                              float alpha, const void* X, int64_t M, void* Y, float* U_save,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+  qlora_status st = check_linear(W, A, B, r, M, X, workspace, workspace_bytes, false);
+  if (st != QLORA_OK) return st;
+  if (M == 0) return QLORA_OK;
+  if (!Y) return QLORA_ERR_NULL;
+  if (!aligned16(Y) || (U_save && !aligned16(U_save))) return QLORA_ERR_ALIGN;
+  return linear_forward(*W, *level_table(W->table), A, B, r, alpha, X, M, Y, U_save, workspace,
+                        static_cast<cudaStream_t>(stream));
+}
+
+qlora_status qlora_linear_bwd(const qlora_nf4* W, const void* A, const void* B, int32_t r,
+                              float alpha, const void* X, const float* U, const void* dY,
+                              int64_t M, void* dX, float* dA, float* dB, int32_t accumulate,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+  qlora_status st = check_linear(W, A, B, r, M, X, workspace, workspace_bytes, true);
+  if (st != QLORA_OK) return st;
+  if ((M > 0 && !dY) || !dA || !dB) return QLORA_ERR_NULL;
+  if (!aligned16(dY) || !aligned16(dA) || !aligned16(dB) || (dX && !aligned16(dX)) ||
+      (U && !aligned16(U)))
+    return QLORA_ERR_ALIGN;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (M == 0) {
+    if (accumulate) return QLORA_OK;
+    // no tokens: the gradients of A and B are zero
+    if (cudaMemsetAsync(dA, 0, sizeof(float) * r * W->cols, s) != cudaSuccess ||
+        cudaMemsetAsync(dB, 0, sizeof(float) * r * W->rows, s) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+    return QLORA_OK;
+  }
+  return linear_backward(*W, *level_table(W->table), A, B, r, alpha, X, U, dY, M, dX, dA, dB,
+                         accumulate != 0, workspace, s);
+}
+
+qlora_status qlora_check(void* workspace, void* stream) {
+  if (!workspace) return QLORA_ERR_NULL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return QLORA_ERR_CUDA;
+  DeviceStatus h{};
+  if (cudaMemcpy(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  if (h.code != 0u) {
+    if (cudaMemset(workspace, 0, sizeof(h)) != cudaSuccess) return QLORA_ERR_CUDA;
+    return static_cast<qlora_status>(h.code);
+  }
+  return QLORA_OK;
+}
+
+uint64_t qlora_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+}  // extern "C"

@@ -1,0 +1,72 @@
+// Internal declarations shared by the translation units of libqlora.so.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "qlora.h"
+
+namespace qlora {
+
+// First 256 bytes of every workspace: a status word written by kernels that
+// detect an error on the device, read (and cleared) by qlora_check().
+constexpr size_t kStatusBytes = 256;
+struct DeviceStatus {
+  unsigned int code;    // qlora_status, first error wins
+  unsigned int detail;  // kernel-specific detail (e.g. which wait gave up)
+};
+
+#ifdef __CUDACC__
+__device__ __forceinline__ void report(DeviceStatus* st, unsigned int code,
+                                       unsigned int detail) {
+  if (st && atomicCAS(&st->code, 0u, code) == 0u) st->detail = detail;
+}
+#endif
+
+// Level table and decision thresholds handed to kernels by value.
+// thr[k] is the largest fp32 not above the exact midpoint of levels k, k+1,
+// so that, for fp32 x, (x > thr[k]) == (x > exact midpoint).
+struct LevelTable {
+  float level[16];
+  float thr[16];  // 15 used
+};
+
+// tables.cpp
+qlora_status make_level_table(int32_t table, LevelTable* out);
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// abi.cu: every kernel launch site calls this once per launch.
+void count_launch(unsigned n = 1);
+
+inline bool aligned16(const void* p) {
+  return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+// quantize.cu
+qlora_status launch_quantize(const void* W, int32_t w_dtype, const qlora_nf4& q,
+                             const LevelTable& t, void* workspace, cudaStream_t s);
+qlora_status launch_dequantize(const qlora_nf4& q, const LevelTable& t, void* out,
+                               int32_t out_dtype, cudaStream_t s);
+
+// Everything a linear-layer kernel needs to read a quantised W.
+struct QView {
+  const uint8_t* codes;
+  const int8_t* scale_codes;
+  const float* factors;
+  const float* mean;
+  int64_t rows, cols;
+  int32_t dq_shift;  // log2(dq_blocksize); -1 without double quantisation
+};
+
+#ifdef __CUDACC__
+__device__ __forceinline__ float block_scale(const QView& w, int64_t b, float mu) {
+  if (w.dq_shift < 0) return __ldg(w.factors + b);
+  float q = static_cast<float>(__ldg(w.scale_codes + b));
+  float f = __ldg(w.factors + (b >> w.dq_shift));
+  return __fadd_rn(__fmul_rn(q, f), mu);
+}
+#endif
+
+}  // namespace qlora

@@ -1,0 +1,235 @@
+"""Python binding of libqlora.so (argument marshalling only).
+
+Every function named ``qlora_*`` here calls the C entry point of the same
+name in ``include/qlora.h``; tensors are torch tensors (device memory and the
+current CUDA stream come from torch), and every step of the computation runs
+in the library's CUDA kernels.  A missing library raises immediately: there
+is no other implementation to fall back to.
+"""
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqlora.so")
+
+QLORA_OK = 0
+QLORA_ERR_NULL = 1
+QLORA_ERR_ALIGN = 2
+QLORA_ERR_SHAPE = 3
+QLORA_ERR_UNSUPPORTED = 4
+QLORA_ERR_NONFINITE = 5
+QLORA_ERR_DEVICE_TIMEOUT = 6
+QLORA_ERR_CUDA = 7
+QLORA_ERR_WORKSPACE = 8
+
+QLORA_F32 = 0
+QLORA_BF16 = 1
+QLORA_TABLE_NF4 = 0
+QLORA_TABLE_UNIFORM = 1
+
+_DTYPE = {torch.float32: QLORA_F32, torch.bfloat16: QLORA_BF16}
+
+
+class qlora_nf4(ctypes.Structure):
+    _fields_ = [
+        ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
+        ("blocksize", ctypes.c_int32), ("dq_blocksize", ctypes.c_int32),
+        ("table", ctypes.c_int32), ("reserved", ctypes.c_int32),
+        ("codes", ctypes.c_void_p), ("scale_codes", ctypes.c_void_p),
+        ("factors", ctypes.c_void_p), ("mean", ctypes.c_void_p),
+    ]
+
+
+class QloraError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = int(status)
+        super().__init__(f"{where}: {qlora_status_string(status)} (status {status})")
+
+
+_lib = None
+
+
+def lib():
+    """Load libqlora.so once; raise if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m bit_nf4_quantized_17_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        i32, i64, sz, vp, f32 = (ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t,
+                                 ctypes.c_void_p, ctypes.c_float)
+        psz = ctypes.POINTER(ctypes.c_size_t)
+        pq = ctypes.POINTER(qlora_nf4)
+        sig = {
+            "qlora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+            "qlora_levels": (ctypes.c_int, [i32, ctypes.POINTER(ctypes.c_float)]),
+            "qlora_nf4_sizes": (ctypes.c_int, [i64, i64, i32, i32, psz, psz, psz, psz, psz]),
+            "qlora_quantize": (ctypes.c_int, [vp, i32, pq, vp, sz, vp]),
+            "qlora_dequantize": (ctypes.c_int, [pq, vp, i32, vp]),
+            "qlora_linear_workspace": (ctypes.c_int, [i64, i64, i64, i32, psz, psz]),
+            "qlora_linear_fwd": (ctypes.c_int, [pq, vp, vp, i32, f32, vp, i64, vp, vp, vp, sz, vp]),
+            "qlora_linear_bwd": (ctypes.c_int, [pq, vp, vp, i32, f32, vp, vp, vp, i64, vp, vp, vp,
+                                                i32, vp, sz, vp]),
+            "qlora_check": (ctypes.c_int, [vp, vp]),
+            "qlora_launch_count": (ctypes.c_uint64, []),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ok(status, where):
+    if status != QLORA_OK:
+        raise QloraError(status, where)
+
+
+def qlora_status_string(status):
+    return lib().qlora_status_string(int(status)).decode()
+
+
+def qlora_levels(table=QLORA_TABLE_NF4):
+    out = (ctypes.c_float * 16)()
+    _ok(lib().qlora_levels(table, out), "qlora_levels")
+    return list(out)
+
+
+def qlora_nf4_sizes(rows, cols, blocksize=64, dq_blocksize=256):
+    vals = [ctypes.c_size_t() for _ in range(5)]
+    _ok(lib().qlora_nf4_sizes(rows, cols, blocksize, dq_blocksize,
+                              *[ctypes.byref(v) for v in vals]), "qlora_nf4_sizes")
+    keys = ("codes", "scale_codes", "factors", "mean", "workspace")
+    return {k: v.value for k, v in zip(keys, vals)}
+
+
+def qlora_linear_workspace(M, N, K, r):
+    f, b = ctypes.c_size_t(), ctypes.c_size_t()
+    _ok(lib().qlora_linear_workspace(M, N, K, r, ctypes.byref(f), ctypes.byref(b)),
+        "qlora_linear_workspace")
+    return f.value, b.value
+
+
+def _workspace(nbytes, device):
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+@dataclass
+class QuantizedWeight:
+    """Caller-owned device arrays of one quantised weight (see qlora_nf4)."""
+    rows: int
+    cols: int
+    blocksize: int
+    dq_blocksize: int
+    table: int
+    codes: torch.Tensor
+    scale_codes: torch.Tensor
+    factors: torch.Tensor
+    mean: torch.Tensor
+
+    @classmethod
+    def empty(cls, rows, cols, blocksize=64, dq_blocksize=256, table=QLORA_TABLE_NF4,
+              device="cuda"):
+        sz = qlora_nf4_sizes(rows, cols, blocksize, dq_blocksize)
+        return cls(rows, cols, blocksize, dq_blocksize, table,
+                   torch.empty(sz["codes"], dtype=torch.uint8, device=device),
+                   torch.empty(max(sz["scale_codes"], 1), dtype=torch.int8, device=device),
+                   torch.empty(sz["factors"] // 4, dtype=torch.float32, device=device),
+                   torch.empty(max(sz["mean"] // 4, 1), dtype=torch.float32, device=device))
+
+    @property
+    def struct(self):
+        return qlora_nf4(self.rows, self.cols, self.blocksize, self.dq_blocksize, self.table, 0,
+                         self.codes.data_ptr(), self.scale_codes.data_ptr(),
+                         self.factors.data_ptr(), self.mean.data_ptr())
+
+    @property
+    def nbytes(self):
+        sz = qlora_nf4_sizes(self.rows, self.cols, self.blocksize, self.dq_blocksize)
+        return sz["codes"] + sz["scale_codes"] + sz["factors"] + sz["mean"]
+
+
+def qlora_quantize(W, blocksize=64, dq_blocksize=256, table=QLORA_TABLE_NF4, out=None,
+                   workspace=None, stream=None, check=True):
+    """Quantise a 2-D fp32/bf16 CUDA tensor; returns a QuantizedWeight."""
+    assert W.is_cuda and W.dim() == 2 and W.is_contiguous() and W.dtype in _DTYPE
+    rows, cols = W.shape
+    q = out or QuantizedWeight.empty(rows, cols, blocksize, dq_blocksize, table, W.device)
+    if workspace is None:
+        workspace = _workspace(qlora_nf4_sizes(rows, cols, blocksize, dq_blocksize)["workspace"],
+                               W.device)
+    st = q.struct
+    _ok(lib().qlora_quantize(_ptr(W), _DTYPE[W.dtype], ctypes.byref(st), _ptr(workspace),
+                             workspace.numel(), _stream(stream)), "qlora_quantize")
+    if check:
+        qlora_check(workspace, stream)
+    return q
+
+
+def qlora_dequantize(q, dtype=torch.float32, out=None, stream=None):
+    out = out if out is not None else torch.empty((q.rows, q.cols), dtype=dtype,
+                                                  device=q.codes.device)
+    st = q.struct
+    _ok(lib().qlora_dequantize(ctypes.byref(st), _ptr(out), _DTYPE[out.dtype], _stream(stream)),
+        "qlora_dequantize")
+    return out
+
+
+def qlora_linear_fwd(q, A, B, alpha, X, Y=None, U_save=None, workspace=None, stream=None):
+    """Y = X W^T + (alpha/r) (X A^T) B^T.  Returns Y (and fills U_save if given)."""
+    M = X.shape[0]
+    r = A.shape[0]
+    if Y is None:
+        Y = torch.empty((M, q.rows), dtype=torch.bfloat16, device=X.device)
+    if workspace is None:
+        workspace = _workspace(qlora_linear_workspace(M, q.rows, q.cols, r)[0], X.device)
+    st = q.struct
+    _ok(lib().qlora_linear_fwd(ctypes.byref(st), _ptr(A), _ptr(B), r, float(alpha), _ptr(X), M,
+                               _ptr(Y), _ptr(U_save), _ptr(workspace), workspace.numel(),
+                               _stream(stream)), "qlora_linear_fwd")
+    return Y
+
+
+def qlora_linear_bwd(q, A, B, alpha, X, U, dY, dX=None, dA=None, dB=None, accumulate=False,
+                     want_dx=True, workspace=None, stream=None):
+    """Returns (dX, dA, dB); W gets no gradient."""
+    M = X.shape[0]
+    r = A.shape[0]
+    dev = X.device
+    if want_dx and dX is None:
+        dX = torch.empty((M, q.cols), dtype=torch.bfloat16, device=dev)
+    if dA is None:
+        dA = torch.empty((r, q.cols), dtype=torch.float32, device=dev)
+    if dB is None:
+        dB = torch.empty((q.rows, r), dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = _workspace(qlora_linear_workspace(M, q.rows, q.cols, r)[1], dev)
+    st = q.struct
+    _ok(lib().qlora_linear_bwd(ctypes.byref(st), _ptr(A), _ptr(B), r, float(alpha), _ptr(X),
+                               _ptr(U), _ptr(dY), M, _ptr(dX) if want_dx else None, _ptr(dA),
+                               _ptr(dB), 1 if accumulate else 0, _ptr(workspace),
+                               workspace.numel(), _stream(stream)), "qlora_linear_bwd")
+    return dX, dA, dB
+
+
+def qlora_launch_count():
+    return int(lib().qlora_launch_count())
+
+
+def qlora_check(workspace, stream=None):
+    _ok(lib().qlora_check(_ptr(workspace), _stream(stream)), "qlora_check")

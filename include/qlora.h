@@ -1,0 +1,164 @@
+/*
+ * qlora.h - C ABI of libqlora.so: a QLoRA linear layer on one B200 (sm_100a).
+ *
+ * The frozen base weight W (d_out x d_in) is stored block-wise in 4 bits:
+ * absmax per block of `blocksize` consecutive weights, the nearest of 16
+ * levels (NF4 or the uniform grid), two indices per byte, and the fp32 block
+ * scales quantised again to int8 ("double quantisation").  The layer adds a
+ * trainable bf16 LoRA branch:
+ *
+ *     forward   Y  = X W^T + s (X A^T) B^T,            s = alpha / r
+ *     backward  dX = dY W + s (dY B) A,  dB = s dY^T (X A^T),  dA = s (dY B)^T X
+ *
+ * with no gradient for W.  Sources (page title, section):
+ *   - quantise / store:  "QLoRA技术从入门到精通", 3(1) 基座模型初始化量化;
+ *                         "LoRA 与 QLoRA：用一块 GPU 微调大模型", 量化 (分块缩放, NF4, 存储和计算)
+ *   - dequantise:         "QLoRA技术从入门到精通", 3(2) 前向传播 (X_deq = grid[idx] * scale)
+ *   - forward:            "LoRA 与 QLoRA：把大模型微调拆成可负担的工程", 2 (h = W x + (α/r) B A x)
+ *   - backward:           "QLoRA技术从入门到精通", 3(3) 反向传播; same page as forward, 6
+ *
+ * Conventions for every call:
+ *   - All matrices are dense row-major.  X: M x d_in, Y and dY: M x d_out,
+ *     A: r x d_in, B: d_out x r, dX: M x d_in (all bf16); U: M x r,
+ *     dA: r x d_in, dB: d_out x r (all fp32).
+ *   - Pointers named "device" are CUDA device pointers, 16-byte aligned.  The
+ *     caller owns and allocates every buffer (sizes from the *_sizes and
+ *     *_workspace queries); the library never allocates, frees or keeps a
+ *     pointer after a call returns.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *     stream-ordered and asynchronous: they return after enqueueing work.
+ *   - Argument errors are found on the host and returned before any launch.
+ *     Errors found on the device (a non-finite weight, a bounded wait that
+ *     gave up) are written to a status word at the start of the workspace;
+ *     qlora_check() synchronises the stream and returns it.
+ *   - No call exits, aborts or traps.
+ */
+#ifndef QLORA_H
+#define QLORA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QLORA_OK = 0,
+  QLORA_ERR_NULL = 1,           /* a required pointer is NULL */
+  QLORA_ERR_ALIGN = 2,          /* a device pointer is not 16-byte aligned */
+  QLORA_ERR_SHAPE = 3,          /* a size is out of range or sizes disagree */
+  QLORA_ERR_UNSUPPORTED = 4,    /* valid request this build does not implement */
+  QLORA_ERR_NONFINITE = 5,      /* quantise met a NaN or an infinity (device status) */
+  QLORA_ERR_DEVICE_TIMEOUT = 6, /* a bounded device-side wait gave up (device status) */
+  QLORA_ERR_CUDA = 7,           /* a CUDA runtime call or launch failed */
+  QLORA_ERR_WORKSPACE = 8       /* workspace missing or smaller than the query said */
+} qlora_status;
+
+typedef enum { QLORA_F32 = 0, QLORA_BF16 = 1 } qlora_dtype;
+
+/* Level tables.  NF4: medians of equal-probability intervals of N(0,1),
+ * 7 below zero, an exact 0, 8 above, each half scaled so the ends are -1 and
+ * +1 ("QLoRA技术从入门到精通", 2(3)2) NF4非均匀格点).  UNIFORM: -1 + k*2/15
+ * ("QLoRA 量化微调", 7.1). */
+typedef enum { QLORA_TABLE_NF4 = 0, QLORA_TABLE_UNIFORM = 1 } qlora_table;
+
+/* A quantised weight.  Block b covers flattened row-major elements
+ * [b*blocksize, (b+1)*blocksize); group g covers blocks [g*dq_blocksize,
+ * (g+1)*dq_blocksize).  n = rows*cols, nb = ceil(n/blocksize),
+ * ng = ceil(nb/dq_blocksize).
+ *   codes        device, ceil(n/2) bytes: element 2j in the low nibble of
+ *                byte j, element 2j+1 in the high nibble
+ *   scale_codes  device, nb int8 (dq_blocksize > 0), else unused (may be NULL)
+ *   factors      device fp32: ng group factors absmax_g/127 (dq_blocksize > 0),
+ *                or the nb block absmax values themselves (dq_blocksize = 0)
+ *   mean         device, 1 fp32: mean of the block scales (dq_blocksize > 0),
+ *                else unused (may be NULL)
+ * Block b dequantises with s_b = fp32(fp32(scale_codes[b] * factors[b/dq]) + mean)
+ * (or factors[b] without double quantisation) and w = fp32(level[idx] * s_b). */
+typedef struct {
+  int64_t rows;          /* d_out */
+  int64_t cols;          /* d_in */
+  int32_t blocksize;     /* 64, 128, 256, 512 or 1024 */
+  int32_t dq_blocksize;  /* 0 (no double quantisation), 64, 128, 256, 512 or 1024 */
+  int32_t table;         /* qlora_table */
+  int32_t reserved;      /* set to 0 */
+  uint8_t* codes;
+  int8_t* scale_codes;
+  float* factors;
+  float* mean;
+} qlora_nf4;
+
+/* Human-readable name of a status code (static storage). */
+const char* qlora_status_string(qlora_status s);
+
+/* The library's own 16 fp32 levels of `table` (host memory, ascending). */
+qlora_status qlora_levels(int32_t table, float levels_out[16]);
+
+/* Byte sizes of the arrays of a quantised rows x cols weight and of the
+ * workspace qlora_quantize needs.  Any output pointer may be NULL.
+ * QLORA_ERR_SHAPE for rows, cols < 1 or more than 2^36 elements;
+ * QLORA_ERR_UNSUPPORTED for a blocksize or dq_blocksize not listed above. */
+qlora_status qlora_nf4_sizes(int64_t rows, int64_t cols, int32_t blocksize,
+                             int32_t dq_blocksize, size_t* codes_bytes,
+                             size_t* scale_codes_bytes, size_t* factors_bytes,
+                             size_t* mean_bytes, size_t* workspace_bytes);
+
+/* Quantise W (device, rows*cols values of w_dtype, row-major) into the arrays
+ * of *q (host struct holding device pointers; rows, cols, blocksize,
+ * dq_blocksize and table describe the request).  Steps: block absmax, divide
+ * (IEEE fp32), nearest level (exact; a value halfway between two levels takes
+ * the lower index), pack; then, with double quantisation, the mean of the
+ * block scales on a fixed-point grid of 2^(E-32) (E = binary exponent of the
+ * largest scale; order-independent), int8 codes of scale - mean per group
+ * with factor absmax/127, round half to even.  A non-finite weight sets
+ * QLORA_ERR_NONFINITE in the workspace status (outputs then undefined).
+ * workspace: device, >= workspace_bytes from qlora_nf4_sizes. */
+qlora_status qlora_quantize(const void* W, int32_t w_dtype, const qlora_nf4* q,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/* Dequantise *q into W_out (device, rows*cols values of out_dtype):
+ * fp32 out is w = fp32(level[idx] * s_b) bit for bit; bf16 out is that value
+ * rounded to nearest even.  Needs no workspace. */
+qlora_status qlora_dequantize(const qlora_nf4* q, void* W_out, int32_t out_dtype,
+                              void* stream);
+
+/* Workspace bytes for qlora_linear_fwd / qlora_linear_bwd at these sizes
+ * (N = d_out, K = d_in).  Either output may be NULL. */
+qlora_status qlora_linear_workspace(int64_t M, int64_t N, int64_t K, int32_t r,
+                                    size_t* fwd_bytes, size_t* bwd_bytes);
+
+/* Forward pass Y = X W^T + s (X A^T) B^T with W dequantised on the fly (a
+ * full-precision W is never written to memory).  Requirements: W->cols % 64
+ * == 0 and W->blocksize == 64 (else QLORA_ERR_UNSUPPORTED), 1 <= r <= 256,
+ * M >= 0 (M = 0 is a no-op).  Device buffers: A (r x K bf16), B (N x r bf16),
+ * X (M x K bf16), Y (M x N bf16, written), U_save (M x r fp32, written with
+ * X A^T; may be NULL), workspace (>= fwd_bytes). */
+qlora_status qlora_linear_fwd(const qlora_nf4* W, const void* A, const void* B,
+                              int32_t r, float alpha, const void* X, int64_t M,
+                              void* Y, float* U_save, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
+/* Backward pass: dX = dY W + s V A, dB = s dY^T U, dA = s V^T X, V = dY B.
+ * W receives no gradient.  U (M x r fp32, from the forward) may be NULL: it is
+ * then recomputed as X A^T.  dX (M x K bf16) may be NULL to skip it.  dA
+ * (r x K fp32) and dB (N x r fp32) are overwritten, or added to when
+ * accumulate != 0.  Same requirements as the forward; workspace >= bwd_bytes. */
+qlora_status qlora_linear_bwd(const qlora_nf4* W, const void* A, const void* B,
+                              int32_t r, float alpha, const void* X, const float* U,
+                              const void* dY, int64_t M, void* dX, float* dA,
+                              float* dB, int32_t accumulate, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
+/* Synchronise `stream`, then return and clear the device status word that
+ * calls given this workspace wrote (QLORA_OK if none). */
+qlora_status qlora_check(void* workspace, void* stream);
+
+/* Number of kernels this library has enqueued since it was loaded (all
+ * threads, all calls; memsets not counted).  Host only, never fails. */
+uint64_t qlora_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QLORA_H */

@@ -1,0 +1,154 @@
+"""GPU parity of the QLoRA linear forward and backward against the oracle.
+
+Forward Y = X W^T + s (X A^T) B^T and backward dX = dY W + s V A,
+dB = s dY^T U, dA = s V^T X (V = dY B), with W the oracle's own dequantised
+weight.  bf16 outputs within the stated tolerance (tests/parity.py); fp32
+U, dA, dB within the same tolerance.  At the full sizes the oracle checks
+sampled token rows of Y and dX and every element of U, dA and dB.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bit_nf4_quantized_17_b200 import qlora as Q
+from bit_nf4_quantized_17_b200 import workloads as WL
+from parity import assert_close, f64
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _w_hat(W_cpu):
+    ref = oracle.quantize(W_cpu.float().numpy(), 64, 256)
+    return oracle.dequantize(ref).reshape(W_cpu.shape)
+
+
+def _run(inp, alpha, rows=None, w_hat=None, check=True):
+    """Run fwd + bwd on the GPU and compare with the oracle (optionally on a
+    subset of token rows for Y and dX)."""
+    W, A, B, X, dY = (inp[k] for k in ("W", "A", "B", "X", "dY"))
+    M, r = X.shape[0], A.shape[0]
+    q = Q.qlora_quantize(W.to(DEV))
+    Ad, Bd, Xd, dYd = (t.to(DEV) for t in (A, B, X, dY))
+    U = torch.empty((M, r), dtype=torch.float32, device=DEV)
+    Y = Q.qlora_linear_fwd(q, Ad, Bd, alpha, Xd, U_save=U)
+    dX, dA, dB = Q.qlora_linear_bwd(q, Ad, Bd, alpha, Xd, U, dYd)
+    torch.cuda.synchronize()
+    if not check:
+        return q, Y, U, dX, dA, dB
+    w_hat = _w_hat(W) if w_hat is None else w_hat
+    a, b, x, dy = f64(A), f64(B), f64(X), f64(dY)
+    sel = slice(None) if rows is None else rows
+    y_ref, _ = oracle.linear_fwd(w_hat, a, b, alpha, x[sel])
+    assert_close(f64(Y)[sel], y_ref, "Y")
+    u_ref = x @ a.T
+    assert_close(U, u_ref, "U")
+    dx_ref, _, _ = oracle.linear_bwd(w_hat, a, b, alpha, x[sel], dy[sel])
+    assert_close(f64(dX)[sel], dx_ref, "dX")
+    s = oracle.lora_scale(alpha, r)
+    v = dy @ b
+    assert_close(dA, s * (v.T @ x), "dA")
+    assert_close(dB, s * (dy.T @ u_ref), "dB")
+    return q, Y, U, dX, dA, dB
+
+
+def _inputs(d_out, d_in, r, M, seed, w_std=0.02, b_std=0.01):
+    shape = WL.LinearShape(d_out, d_in, r, 2.0 * r, w_std=w_std)
+    inp = WL.linear_inputs(shape, M, seed)
+    if b_std != 0.01:
+        inp["B"] = WL.randn((d_out, r), b_std, seed + 2, torch.bfloat16)
+    return inp, shape.alpha
+
+
+def test_single_linear_256():
+    shape = WL.WORKLOADS["single_256"].linears[0]
+    _run(WL.linear_inputs(shape, 16, 0), shape.alpha)
+
+
+@pytest.mark.parametrize("M,N,K,r", [
+    (1, 64, 64, 1), (3, 80, 192, 5), (17, 200, 128, 16), (130, 96, 320, 64),
+    (257, 384, 256, 8), (64, 128, 4096, 256), (300, 1000, 640, 24),
+])
+def test_ragged_shapes(M, N, K, r):
+    inp, alpha = _inputs(N, K, r, M, 1000 + M, b_std=0.05)
+    _run(inp, alpha)
+
+
+@pytest.fixture(scope="module")
+def attn():
+    shape = WL.WORKLOADS["attn_4096"].linears[0]
+    inp = WL.linear_inputs(shape, 4096, 0)
+    return shape, inp, _w_hat(inp["W"])
+
+
+def test_attention_projection_4096(attn):
+    shape, inp, w_hat = attn
+    rows = np.sort(np.random.default_rng(0).choice(4096, 96, replace=False))
+    rows = np.concatenate([[0], rows, [4095]])
+    _run(inp, shape.alpha, rows=rows, w_hat=w_hat)
+
+
+@pytest.fixture(scope="module", params=[0, 1], ids=["gate_up", "down"])
+def mlp(request):
+    shape = WL.WORKLOADS["mlp_11008"].linears[request.param]
+    W = WL.weight(shape, 16 * request.param)
+    return shape, request.param, W, _w_hat(W)
+
+
+@pytest.mark.parametrize("M", [1, 16, 8192])
+def test_mlp_shapes(mlp, M):
+    shape, j, W, w_hat = mlp
+    seed = 16 * j
+    inp = dict(W=W, A=WL.lora_a(shape, seed), B=WL.lora_b(shape, seed),
+               X=WL.activations(shape, M, seed), dY=WL.grad_output(shape, M, seed))
+    rows = None
+    if M > 64:
+        rows = np.sort(np.random.default_rng(M).choice(M, 64, replace=False))
+        rows = np.concatenate([[0], rows, [M - 1]])
+    _run(inp, shape.alpha, rows=rows, w_hat=w_hat)
+
+
+def test_zero_b_gives_base_output():
+    inp, alpha = _inputs(192, 256, 8, 33, 7)
+    inp["B"] = torch.zeros_like(inp["B"])
+    q, Y, U, dX, dA, dB = _run(inp, alpha)
+    base = f64(inp["X"]) @ _w_hat(inp["W"]).astype(np.float64).T
+    assert_close(Y, base, "Y(B=0)")
+    assert torch.count_nonzero(dA) == 0
+
+
+def test_accumulate_recompute_skip_and_determinism():
+    inp, alpha = _inputs(320, 384, 16, 70, 11, b_std=0.05)
+    q, Y, U, dX, dA, dB = _run(inp, alpha)
+    A, B, X, dY = (inp[k].to(DEV) for k in ("A", "B", "X", "dY"))
+    # same inputs again: bit-identical outputs
+    Y2 = Q.qlora_linear_fwd(q, A, B, alpha, X)
+    assert torch.equal(Y, Y2)
+    # U recomputed inside the backward when not given
+    dX2, dA2, dB2 = Q.qlora_linear_bwd(q, A, B, alpha, X, None, dY)
+    assert torch.equal(dX, dX2) and torch.equal(dA, dA2) and torch.equal(dB, dB2)
+    # accumulate adds onto the given gradients
+    dA3, dB3 = dA.clone(), dB.clone()
+    Q.qlora_linear_bwd(q, A, B, alpha, X, U, dY, dA=dA3, dB=dB3, accumulate=True)
+    torch.cuda.synchronize()
+    assert torch.equal(dA3, dA + dA) and torch.equal(dB3, dB + dB)
+    # dX may be skipped
+    _, dA4, dB4 = Q.qlora_linear_bwd(q, A, B, alpha, X, U, dY, want_dx=False)
+    assert torch.equal(dA4, dA) and torch.equal(dB4, dB)
+
+
+def test_zero_tokens():
+    inp, alpha = _inputs(128, 128, 8, 1, 3)
+    q = Q.qlora_quantize(inp["W"].to(DEV))
+    A, B = inp["A"].to(DEV), inp["B"].to(DEV)
+    X = torch.empty((0, 128), dtype=torch.bfloat16, device=DEV)
+    Y = Q.qlora_linear_fwd(q, A, B, alpha, X)
+    assert Y.shape == (0, 128)
+    dA = torch.full((8, 128), 5.0, device=DEV)
+    dB = torch.full((128, 8), 5.0, device=DEV)
+    Q.qlora_linear_bwd(q, A, B, alpha, X, None, torch.empty((0, 128), dtype=torch.bfloat16,
+                                                            device=DEV), dA=dA, dB=dB)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(dA) == 0 and torch.count_nonzero(dB) == 0
