@@ -1,6 +1,8 @@
 // C ABI of libqlora.so: argument checks on the host, then kernel launches on
 // the caller's stream.  See include/qlora.h for the contract of each call.
 #include <atomic>
+#include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -15,6 +17,20 @@ std::atomic<uint64_t> g_launches{0};
 }  // namespace
 
 void qlora::count_launch(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+qlora_status qlora::after_launch(const char* kernel, cudaStream_t s) {
+  static const bool sync_check = [] {
+    const char* e = std::getenv("QLORA_SYNC_CHECK");
+    return e && e[0] == '1';
+  }();
+  cudaError_t e = cudaPeekAtLastError();
+  if (e == cudaSuccess && sync_check) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) {
+    if (sync_check) std::fprintf(stderr, "qlora: %s: %s\n", kernel, cudaGetErrorString(e));
+    return QLORA_ERR_CUDA;
+  }
+  return QLORA_OK;
+}
 
 namespace {
 

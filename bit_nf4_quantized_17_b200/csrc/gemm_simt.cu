@@ -37,7 +37,8 @@ __device__ __forceinline__ float load_operand(const Operand& o, int64_t i, int64
     const int64_t e = row * o.w.cols + col;
     const uint8_t byte = __ldg(o.w.codes + (e >> 1));
     const int idx = (e & 1) ? (byte >> 4) : (byte & 15);
-    return __fmul_rn(lv[idx], block_scale(o.w, e >> 6, mu));
+    // the product uses the dequantised weight rounded to bf16
+    return __bfloat162float(__float2bfloat16_rn(__fmul_rn(lv[idx], block_scale(o.w, e >> 6, mu))));
   }
 }
 
@@ -123,7 +124,7 @@ qlora_status simt_gemm(int kind_a, const Operand& a, int kind_b, const Operand& 
   QLORA_CASE(OP_F32_MN, OP_BF16_MN)
   { return QLORA_ERR_UNSUPPORTED; }
 #undef QLORA_CASE
-  return cudaPeekAtLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  return after_launch("simt_gemm", s);
 }
 
 }  // namespace qlora

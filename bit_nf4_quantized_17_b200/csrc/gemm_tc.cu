@@ -1,0 +1,618 @@
+// Tensor-core (tcgen05 / TMEM / TMA) contractions of the QLoRA linear layer.
+//
+// One warp-specialised kernel computes a 128-row tile D[m0:m0+128, n0:n0+bn]
+// of D = A . B^T with fp32 accumulation in TMEM:
+//
+//   warp 0      TMA producer: A tiles (bf16, K- or MN-major, 128B swizzle),
+//               and either B tiles (bf16) or the packed 4-bit codes of W
+//   warp 1      allocates TMEM; one thread issues tcgen05.mma (M=128, N=bn,
+//               K=16) and commits each stage back to the producer
+//   warps 4-11  dequantise W on load (modes B_DQ_*): per 64-weight block
+//               they build the 16 bf16 values fp32(level[k] * s_hat) of the
+//               block's own table and expand every nibble with byte permutes
+//               straight into the 128B-swizzled bf16 B tile; then they drain
+//               the accumulator from TMEM and store the tile
+//
+// After the main loop optional "extension" stages append a second pair of
+// bf16 operands along K (A2, B2): this is how the rank-r LoRA term
+// s (X A^T) B^T (forward) or s (dY B) A (backward dX) is added into the same
+// accumulator as the dequantised-weight product, so Y and dX leave the kernel
+// once, in bf16, and the full-precision W never exists outside shared memory
+// ("QLoRA技术从入门到精通", 3(2): dequantise one layer at a time and discard).
+//
+// Every mbarrier wait is bounded; a wait that gives up raises a CTA-wide
+// abort, the kernel drains its own copies and MMAs, frees TMEM and reports
+// QLORA_ERR_DEVICE_TIMEOUT in the workspace status word.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+
+#include "internal.cuh"
+#include "kernels.cuh"
+#include "tc_ptx.cuh"
+
+namespace qlora {
+namespace {
+
+constexpr int kThreads = 384;
+constexpr int kABytes = 16384;   // 128 rows x 64 bf16
+constexpr int kCodeBytes = 8192;  // 256 W rows x 32 B (fwd) or 64 W rows x 128 B (bwd)
+constexpr long long kTimeoutCycles = 4000000000ll;  // ~2 s at 1.9 GHz
+
+struct TcArgs {
+  int32_t m, n, bn;
+  int32_t k_tiles;        // main-loop stages per CTA (per split)
+  int32_t kt_total;       // main-loop stages of the whole contraction
+  int32_t k2_tiles;       // extension stages: two halves of k2_half stages each
+  int32_t k2_half;        // stages per half (64 LoRA ranks each)
+  int32_t k2_last_steps;  // K=16 steps in the last stage of each half
+  int32_t a_mn, b2_mn;
+  int32_t b_bytes, stage_bytes, tmem_cols;
+  QView w;
+  int32_t kblocks;        // W.cols / 64
+  float alpha;
+  void* out;
+  int64_t ldo;
+  int32_t out_bf16;
+  int64_t split_stride;
+  int64_t out_elems;      // elements of `out` (stores beyond it are reported, not made)
+  int64_t nblocks;        // entries of w.scale_codes (loads beyond it are reported)
+  DeviceStatus* st;
+};
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Expand 8 nibbles (weights k..k+7, nibble j = weight k+j) into 8 bf16 values
+// T[idx] using the byte tables L (low bytes of T[0..15]) and H (high bytes).
+__device__ __forceinline__ uint4 expand8(uint32_t x, const uint32_t (&L)[4],
+                                         const uint32_t (&H)[4]) {
+  const uint32_t sel = x & 0x77777777u;                          // byte index within a half table
+  const uint32_t msel = ((x >> 1) & 0x44444444u) | 0x32103210u;  // pick the half by bit 3
+  uint4 out;
+  {
+    const uint32_t lo = __byte_perm(__byte_perm(L[0], L[1], sel), __byte_perm(L[2], L[3], sel), msel);
+    const uint32_t hi = __byte_perm(__byte_perm(H[0], H[1], sel), __byte_perm(H[2], H[3], sel), msel);
+    out.x = __byte_perm(lo, hi, 0x5140);
+    out.y = __byte_perm(lo, hi, 0x7362);
+  }
+  {
+    const uint32_t s2 = sel >> 16, m2 = msel >> 16;
+    const uint32_t lo = __byte_perm(__byte_perm(L[0], L[1], s2), __byte_perm(L[2], L[3], s2), m2);
+    const uint32_t hi = __byte_perm(__byte_perm(H[0], H[1], s2), __byte_perm(H[2], H[3], s2), m2);
+    out.z = __byte_perm(lo, hi, 0x5140);
+    out.w = __byte_perm(lo, hi, 0x7362);
+  }
+  return out;
+}
+
+// The 16 dequantised values of one block, bf16(fp32(level[k] * s)), as byte tables.
+__device__ __forceinline__ void block_tables(const float (&lv)[16], float s, uint32_t (&L)[4],
+                                             uint32_t (&H)[4]) {
+  uint32_t P[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) P[j] = pack_bf16x2(__fmul_rn(lv[2 * j], s), __fmul_rn(lv[2 * j + 1], s));
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    L[j] = __byte_perm(P[2 * j], P[2 * j + 1], 0x6420);
+    H[j] = __byte_perm(P[2 * j], P[2 * j + 1], 0x7531);
+  }
+}
+
+__device__ __forceinline__ void store16(const TcArgs& p, int64_t row, int64_t col,
+                                        const uint32_t (&r)[16]) {
+  if (row >= p.m) return;
+  const int64_t base = static_cast<int64_t>(blockIdx.z) * p.split_stride + row * p.ldo + col;
+  const int64_t span = (p.n - col < 16) ? (p.n - col) : 16;
+  if (base < 0 || base + span > p.out_elems) {
+    report(p.st, QLORA_ERR_SHAPE, 200u);
+    return;
+  }
+  if (p.out_bf16) {
+    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + base;
+    if (col + 16 <= p.n) {
+      uint32_t w[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        w[j] = pack_bf16x2(p.alpha * __uint_as_float(r[2 * j]), p.alpha * __uint_as_float(r[2 * j + 1]));
+      reinterpret_cast<uint4*>(o)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+      reinterpret_cast<uint4*>(o)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    } else {
+      for (int j = 0; j < 16 && col + j < p.n; ++j)
+        o[j] = __float2bfloat16_rn(p.alpha * __uint_as_float(r[j]));
+    }
+  } else {
+    float* o = static_cast<float*>(p.out) + base;
+    if (col + 16 <= p.n) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        reinterpret_cast<float4*>(o)[j] =
+            make_float4(p.alpha * __uint_as_float(r[4 * j]), p.alpha * __uint_as_float(r[4 * j + 1]),
+                        p.alpha * __uint_as_float(r[4 * j + 2]), p.alpha * __uint_as_float(r[4 * j + 3]));
+    } else {
+      for (int j = 0; j < 16 && col + j < p.n; ++j) o[j] = p.alpha * __uint_as_float(r[j]);
+    }
+  }
+}
+
+template <int BMODE, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+               const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
+               const TcArgs p, const LevelTable tab) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* full_tma = reinterpret_cast<uint64_t*>(smem + STAGES * p.stage_bytes);
+  uint64_t* full_b = full_tma + STAGES;
+  uint64_t* empty = full_b + STAGES;
+  uint64_t* accum = empty + STAGES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.y * 128;
+  const int n0 = blockIdx.x * p.bn;
+  const int kt0 = blockIdx.z * p.k_tiles;
+  const int k_tiles = min(p.k_tiles, p.kt_total - kt0);
+  const int total = k_tiles + p.k2_tiles;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      ptx::mbar_init(&full_tma[s], 1);
+      ptx::mbar_init(&full_b[s], 256);
+      ptx::mbar_init(&empty[s], 1);
+    }
+    ptx::mbar_init(accum, 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+    ptx::prefetch_tmap(&tmA);
+    ptx::prefetch_tmap(&tmB);
+    if (p.k2_tiles) {
+      ptx::prefetch_tmap(&tmA2);
+      ptx::prefetch_tmap(&tmB2);
+    }
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(tmem_slot, p.tmem_cols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------ TMA producer
+    int issued = 0;
+    for (int kt = 0; kt < total; ++kt) {
+      const int s = kt % STAGES;
+      const uint32_t ph = (kt / STAGES) & 1;
+      if (!ptx::mbar_wait(&empty[s], ph ^ 1, kTimeoutCycles, abort_flag)) break;
+      uint8_t* sa = smem + s * p.stage_bytes;
+      uint8_t* sb = sa + kABytes;
+      uint8_t* sc = sb + p.b_bytes;
+      if (kt < k_tiles) {
+        const int kg = kt0 + kt;
+        const uint32_t bytes = kABytes + (BMODE == B_TMA_K ? p.bn * 128 : kCodeBytes);
+        ptx::mbar_arrive_expect_tx(&full_tma[s], bytes);
+        if (p.a_mn) {
+          ptx::tma_load_2d(&tmA, &full_tma[s], sa, m0, kg * 64);
+          ptx::tma_load_2d(&tmA, &full_tma[s], sa + 8192, m0 + 64, kg * 64);
+        } else {
+          ptx::tma_load_2d(&tmA, &full_tma[s], sa, kg * 64, m0);
+        }
+        if (BMODE == B_TMA_K)
+          ptx::tma_load_2d(&tmB, &full_tma[s], sb, kg * 64, n0);
+        else if (BMODE == B_DQ_K)
+          ptx::tma_load_2d(&tmB, &full_tma[s], sc, kg * 32, n0);
+        else
+          ptx::tma_load_2d(&tmB, &full_tma[s], sc, n0 / 2, kg * 64);
+      } else {
+        // extension stage tt: A2 columns [64 tt, 64 tt + 64) of [hi | lo], B2 ranks
+        // [64 (tt mod half), ...): both halves multiply the same B2 tiles
+        const int tt = kt - k_tiles;
+        const int k2a = tt * 64;
+        const int k2b = (tt % p.k2_half) * 64;
+        ptx::mbar_arrive_expect_tx(&full_tma[s], kABytes + 32768);
+        ptx::tma_load_2d(&tmA2, &full_tma[s], sa, k2a, m0);
+        if (p.b2_mn) {
+#pragma unroll
+          for (int h = 0; h < 4; ++h) ptx::tma_load_2d(&tmB2, &full_tma[s], sb + h * 8192, n0 + 64 * h, k2b);
+        } else {
+          ptx::tma_load_2d(&tmB2, &full_tma[s], sb, k2b, n0);
+        }
+      }
+      ++issued;
+    }
+    // never leave with copies in flight into this CTA's shared memory
+    for (int kt = max(0, issued - STAGES); kt < issued; ++kt)
+      ptx::mbar_wait(&full_tma[kt % STAGES], (kt / STAGES) & 1, kTimeoutCycles, nullptr);
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------ MMA issuer
+    const uint32_t idesc = ptx::idesc_bf16(128, p.bn, p.a_mn, BMODE == B_DQ_MN ? 1 : 0);
+    const uint32_t idesc2 = ptx::idesc_bf16(128, p.bn, 0, p.b2_mn);
+    for (int kt = 0; kt < total; ++kt) {
+      const int s = kt % STAGES;
+      const uint32_t ph = (kt / STAGES) & 1;
+      if (!ptx::mbar_wait(&full_tma[s], ph, kTimeoutCycles, abort_flag)) break;
+      const bool ext = kt >= k_tiles;
+      if (BMODE != B_TMA_K && !ext && !ptx::mbar_wait(&full_b[s], ph, kTimeoutCycles, abort_flag))
+        break;
+      ptx::tc_fence_after();
+      const uint32_t a_addr = ptx::smem_u32(smem + s * p.stage_bytes);
+      const uint32_t b_addr = a_addr + kABytes;
+      const bool a_mn = !ext && p.a_mn;
+      const bool b_mn = ext ? (p.b2_mn != 0) : (BMODE == B_DQ_MN);
+      const int steps = (ext && ((kt - k_tiles) % p.k2_half) == p.k2_half - 1) ? p.k2_last_steps : 4;
+      for (int ks = 0; ks < steps; ++ks) {
+        const uint64_t ad = a_mn ? ptx::sw128_desc(a_addr + ks * 2048, 8192, 1024)
+                                 : ptx::sw128_desc(a_addr + ks * 32, 16, 1024);
+        const uint64_t bd = b_mn ? ptx::sw128_desc(b_addr + ks * 2048, 8192, 1024)
+                                 : ptx::sw128_desc(b_addr + ks * 32, 16, 1024);
+        ptx::umma_bf16(tmem, ad, bd, ext ? idesc2 : idesc, (kt | ks) != 0 ? 1u : 0u);
+      }
+      ptx::umma_commit(&empty[s]);
+    }
+    ptx::umma_commit(accum);
+    ptx::mbar_wait(accum, 0, kTimeoutCycles, nullptr);  // MMAs done before TMEM is freed
+  } else if (warp >= 4) {
+    const int td = threadIdx.x - 128;
+    if (BMODE != B_TMA_K) {
+      // ---------------------------------------------------- dequantisation
+      float lv[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) lv[j] = tab.level[j];
+      const float mu = (p.w.dq_shift >= 0) ? __ldg(p.w.mean) : 0.0f;
+      int row, q;            // row of the codes tile, block within the row
+      int64_t wrow, kb;      // W row and 64-block column of this thread's block
+      if (BMODE == B_DQ_K) {
+        row = td;
+        q = 0;
+      } else {
+        row = td >> 2;
+        q = td & 3;
+      }
+      for (int kt = 0; kt < k_tiles; ++kt) {
+        const int s = kt % STAGES;
+        const uint32_t ph = (kt / STAGES) & 1;
+        const int kg = kt0 + kt;
+        if (BMODE == B_DQ_K) {
+          wrow = n0 + row;
+          kb = kg;
+        } else {
+          wrow = static_cast<int64_t>(kg) * 64 + row;
+          kb = n0 / 64 + q;
+        }
+        bool valid = wrow < p.w.rows && kb < p.kblocks;
+        if (valid && (wrow * p.kblocks + kb >= p.nblocks)) {
+          report(p.st, QLORA_ERR_SHAPE, 201u);
+          valid = false;
+        }
+        const float sc = valid ? block_scale(p.w, wrow * p.kblocks + kb, mu) : 0.0f;
+        if (!ptx::mbar_wait(&full_tma[s], ph, kTimeoutCycles, abort_flag)) break;
+        uint8_t* sa = smem + s * p.stage_bytes;
+        uint8_t* sb = sa + kABytes;
+        const uint8_t* sc_codes = sb + p.b_bytes;
+        const uint8_t* src = (BMODE == B_DQ_K) ? sc_codes + row * 32 : sc_codes + row * 128 + q * 32;
+        const int h0 = (BMODE == B_DQ_K) ? ((row >> 2) & 1) : (row & 1);
+        // the two 16-byte halves are read in an order that spreads banks
+        const uint4 first = *reinterpret_cast<const uint4*>(src + 16 * h0);
+        const uint4 second = *reinterpret_cast<const uint4*>(src + 16 * (h0 ^ 1));
+        uint4 cw[2];
+        cw[0] = h0 ? second : first;
+        cw[1] = h0 ? first : second;
+        uint32_t L[4], H[4];
+        block_tables(lv, sc, L, H);
+        uint32_t words[8] = {cw[0].x, cw[0].y, cw[0].z, cw[0].w,
+                             cw[1].x, cw[1].y, cw[1].z, cw[1].w};
+        if (BMODE == B_DQ_MN) {
+          // threads of one row write different chunks at the same time (bank
+          // spread): word j of this thread becomes chunk (j + 2q) mod 8
+          uint32_t t8[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) t8[j] = (q & 1) ? words[(j + 2) & 7] : words[j];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) words[j] = (q & 2) ? t8[(j + 4) & 7] : t8[j];
+        }
+        uint8_t* dst_row = (BMODE == B_DQ_K) ? sb + row * 128 : sb + q * 8192 + row * 128;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int c = (BMODE == B_DQ_K) ? j : ((j + 2 * q) & 7);
+          const uint4 v = valid ? expand8(words[j], L, H) : make_uint4(0u, 0u, 0u, 0u);
+          *reinterpret_cast<uint4*>(dst_row + 16 * (c ^ (row & 7))) = v;
+        }
+        ptx::fence_proxy_async_smem();
+        ptx::mbar_arrive(&full_b[s]);
+      }
+    }
+    // ---------------------------------------------------------- epilogue
+    bool ok = ptx::mbar_wait(accum, 0, kTimeoutCycles, abort_flag);
+    ok = __all_sync(0xffffffffu, ok && !*abort_flag);
+    if (ok) {
+      ptx::tc_fence_after();
+      const int quarter = warp & 3;
+      const int group = (warp - 4) >> 2;
+      const int64_t row = static_cast<int64_t>(m0) + 32 * quarter + lane;
+      const int nchunks = p.bn / 16;
+      for (int c = group; c < nchunks; c += 2) {
+        uint32_t r[16];
+        ptx::tmem_ld_x16(tmem + (static_cast<uint32_t>(32 * quarter) << 16) + c * 16, r);
+        ptx::tmem_ld_wait();
+        store16(p, row, static_cast<int64_t>(n0) + c * 16, r);
+      }
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, p.tmem_cols);
+  }
+  if (threadIdx.x == 0 && *abort_flag) report(p.st, QLORA_ERR_DEVICE_TIMEOUT, 100u + BMODE);
+}
+
+// Deterministic split-K reduction.  v = sum_z part[z][i][j] (+ part[z][i][j + lo]
+// when lo > 0), summed in a fixed order; then up to three outputs:
+//   o1  fp32  a1 * v, at [i][j] or transposed [j][i], optionally added to o1
+//   o2  bf16  hi = bf16(a2 v) at [i][j] and, if o2_lo > 0, lo = bf16(a2 v - hi) at [i][j + o2_lo]
+//   o3  bf16  the same pair transposed: hi at [j][i], lo at [j + o3_lo][i]
+// hi + lo carries a2 v to about 16 significant bits through bf16 tensor-core operands.
+__global__ void splitk_reduce_kernel(const float* __restrict__ part, int splits, int64_t rows,
+                                     int cols, int pcols, int lo, float* o1, int64_t ld1,
+                                     int trans1, float a1, int acc1, __nv_bfloat16* o2, int64_t ld2,
+                                     float a2, int o2_lo, __nv_bfloat16* o3, int64_t ld3, float a3,
+                                     int o3_lo) {
+  const int64_t total = rows * cols;
+  const int64_t split_stride = rows * pcols;
+  for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t i = e / cols;
+    const int j = static_cast<int>(e - i * cols);
+    const float* src = part + i * pcols + j;
+    float v = 0.0f;
+    for (int z = 0; z < splits; ++z) {
+      v += src[z * split_stride];
+      if (lo) v += src[z * split_stride + lo];
+    }
+    if (o1) {
+      float* dst = trans1 ? o1 + j * ld1 + i : o1 + i * ld1 + j;
+      *dst = acc1 ? *dst + a1 * v : a1 * v;
+    }
+    if (o2) {
+      const float x = a2 * v;
+      const __nv_bfloat16 h = __float2bfloat16_rn(x);
+      o2[i * ld2 + j] = h;
+      if (o2_lo) o2[i * ld2 + j + o2_lo] = __float2bfloat16_rn(x - __bfloat162float(h));
+    }
+    if (o3) {
+      const float x = a3 * v;
+      const __nv_bfloat16 h = __float2bfloat16_rn(x);
+      o3[j * ld3 + i] = h;
+      if (o3_lo) o3[(j + o3_lo) * ld3 + i] = __float2bfloat16_rn(x - __bfloat162float(h));
+    }
+  }
+}
+
+// out[j][i] = hi = bf16(in[i][j]) and, if lo_rows > 0, out[j + lo_rows][i] =
+// bf16(in[i][j] - hi), for a rows x cols fp32 or bf16 matrix.
+template <typename T>
+__global__ void transpose_bf16_kernel(const T* __restrict__ in, int64_t rows, int cols,
+                                      int64_t ld_in, __nv_bfloat16* __restrict__ out,
+                                      int64_t ld_out, int lo_rows) {
+  const int64_t total = rows * cols;
+  for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t i = e / cols;
+    const int j = static_cast<int>(e - i * cols);
+    float v;
+    if constexpr (sizeof(T) == 4)
+      v = in[i * ld_in + j];
+    else
+      v = __bfloat162float(in[i * ld_in + j]);
+    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+    out[j * ld_out + i] = h;
+    if (lo_rows) out[(j + lo_rows) * ld_out + i] = __float2bfloat16_rn(v - __bfloat162float(h));
+  }
+}
+
+// ----------------------------------------------------------------- host
+
+using EncodeFn = PFN_cuTensorMapEncodeTiled_v12000;
+
+EncodeFn encode_fn() {
+  static EncodeFn fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<EncodeFn>(nullptr);
+    return reinterpret_cast<EncodeFn>(f);
+  }();
+  return fn;
+}
+
+// 2-D map over a row-major matrix: `inner` contiguous elements per row, `outer`
+// rows `ld` elements apart; box = box_inner x box_outer elements.
+bool make_map(CUtensorMap* map, const void* base, bool bf16, uint64_t inner, uint64_t outer,
+              uint64_t ld, uint32_t box_inner, uint32_t box_outer, bool swizzle) {
+  EncodeFn enc = encode_fn();
+  if (!enc) return false;
+  const int es = bf16 ? 2 : 1;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {ld * es};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+                   const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int pow2_cols(int bn) {
+  int c = 32;
+  while (c < bn) c <<= 1;
+  return c;
+}
+
+template <int BMODE, int STAGES>
+qlora_status launch_tc(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2,
+                       const CUtensorMap& b2, TcArgs p, const LevelTable& t, dim3 grid,
+                       cudaStream_t s) {
+  const size_t smem = 1024 + static_cast<size_t>(STAGES) * p.stage_bytes + 256;
+  static bool configured = false;
+  if (!configured) {
+    if (cudaFuncSetAttribute(tc_gemm_kernel<BMODE, STAGES>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(232448)) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+    configured = true;
+  }
+  count_launch();
+  tc_gemm_kernel<BMODE, STAGES><<<grid, kThreads, smem, s>>>(a, b, a2, b2, p, t);
+  return after_launch(BMODE == B_TMA_K ? "tc_gemm(lora)" : BMODE == B_DQ_K ? "tc_gemm(fwd)" : "tc_gemm(dgrad)", s);
+}
+
+TcArgs base_args(int m, int n, int bn, DeviceStatus* st) {
+  TcArgs p{};
+  p.m = m;
+  p.n = n;
+  p.bn = bn;
+  p.k2_last_steps = 4;
+  p.k2_half = 1;
+  p.tmem_cols = pow2_cols(bn);
+  p.alpha = 1.0f;
+  p.st = st;
+  return p;
+}
+
+}  // namespace
+
+int tc_split_count(int64_t m_tiles, int64_t k_tiles) {
+  int64_t s = (2 * 148 + m_tiles - 1) / m_tiles;
+  const int64_t max_s = k_tiles / 4 > 0 ? k_tiles / 4 : 1;
+  if (s > max_s) s = max_s;
+  if (s < 1) s = 1;
+  const int64_t per = (k_tiles + s - 1) / s;
+  return static_cast<int>((k_tiles + per - 1) / per);
+}
+
+qlora_status tc_fused_forward(const QView& w, const LevelTable& t, const void* X, int64_t M,
+                              const void* sU, const void* B, int32_t r, void* Y,
+                              DeviceStatus* st, cudaStream_t s) {
+  const int64_t N = w.rows, K = w.cols;
+  CUtensorMap ma, mb, ma2, mb2;
+  if (!make_map(&ma, X, true, K, M, K, 64, 128, true) ||
+      !make_map(&mb, w.codes, false, K / 2, N, K / 2, 32, 256, false) ||
+      !make_map(&ma2, sU, true, 2 * lora_span(r), M, 2 * lora_span(r), 64, 128, true) ||
+      !make_map(&mb2, B, true, r, N, r, 64, 256, true))
+    return QLORA_ERR_CUDA;
+  TcArgs p = base_args(static_cast<int>(M), static_cast<int>(N), 256, st);
+  p.k_tiles = p.kt_total = static_cast<int>(K / 64);
+  p.k2_half = (r + 63) / 64;
+  p.k2_tiles = 2 * p.k2_half;
+  p.k2_last_steps = ((r - 64 * (p.k2_half - 1)) + 15) / 16;
+  p.b_bytes = 32768;
+  p.stage_bytes = kABytes + 32768 + kCodeBytes;
+  p.w = w;
+  p.kblocks = static_cast<int>(K / 64);
+  p.out = Y;
+  p.ldo = N;
+  p.out_bf16 = 1;
+  p.out_elems = M * N;
+  p.nblocks = N * K / 64;
+  dim3 grid(static_cast<unsigned>(ceil_div(N, 256)), static_cast<unsigned>(ceil_div(M, 128)), 1);
+  return launch_tc<B_DQ_K, 3>(ma, mb, ma2, mb2, p, t, grid, s);
+}
+
+qlora_status tc_fused_dgrad(const QView& w, const LevelTable& t, const void* dY, int64_t M,
+                            const void* sV, const void* A, int32_t r, void* dX,
+                            DeviceStatus* st, cudaStream_t s) {
+  const int64_t N = w.rows, K = w.cols;
+  CUtensorMap ma, mb, ma2, mb2;
+  if (!make_map(&ma, dY, true, N, M, N, 64, 128, true) ||
+      !make_map(&mb, w.codes, false, K / 2, N, K / 2, 128, 64, false) ||
+      !make_map(&ma2, sV, true, 2 * lora_span(r), M, 2 * lora_span(r), 64, 128, true) ||
+      !make_map(&mb2, A, true, K, r, K, 64, 64, true))
+    return QLORA_ERR_CUDA;
+  TcArgs p = base_args(static_cast<int>(M), static_cast<int>(K), 256, st);
+  p.k_tiles = p.kt_total = static_cast<int>(ceil_div(N, 64));
+  p.k2_half = (r + 63) / 64;
+  p.k2_tiles = 2 * p.k2_half;
+  p.k2_last_steps = ((r - 64 * (p.k2_half - 1)) + 15) / 16;
+  p.b2_mn = 1;
+  p.b_bytes = 32768;
+  p.stage_bytes = kABytes + 32768 + kCodeBytes;
+  p.w = w;
+  p.kblocks = static_cast<int>(K / 64);
+  p.out = dX;
+  p.ldo = K;
+  p.out_bf16 = 1;
+  p.out_elems = M * K;
+  p.nblocks = N * K / 64;
+  dim3 grid(static_cast<unsigned>(ceil_div(K, 256)), static_cast<unsigned>(ceil_div(M, 128)), 1);
+  return launch_tc<B_DQ_MN, 3>(ma, mb, ma2, mb2, p, t, grid, s);
+}
+
+// part[z] (m_rows x n_cols fp32) = A . B^T over split z of the contraction; A is
+// m_rows x kdim (K-major, or MN-major: stored kdim x m_rows), B is b_rows x kdim
+// K-major (ld_b), read as n_cols rows (a multiple of 16; rows past b_rows are zero).
+qlora_status tc_lora_gemm(const void* A, bool a_mn, int64_t m_rows, int64_t kdim, int64_t ld_a,
+                          const void* B, int64_t ld_b, int32_t b_rows, int32_t n_cols,
+                          float* part, int splits, DeviceStatus* st, cudaStream_t s) {
+  const int bn = n_cols < 256 ? n_cols : 256;
+  CUtensorMap ma, mb;
+  bool ok = a_mn ? make_map(&ma, A, true, m_rows, kdim, ld_a, 64, 64, true)
+                 : make_map(&ma, A, true, kdim, m_rows, ld_a, 64, 128, true);
+  ok = ok && make_map(&mb, B, true, kdim, b_rows, ld_b, 64, bn, true);
+  if (!ok) return QLORA_ERR_CUDA;
+  TcArgs p = base_args(static_cast<int>(m_rows), n_cols, bn, st);
+  p.kt_total = static_cast<int>(ceil_div(kdim, 64));
+  p.k_tiles = static_cast<int>(ceil_div(p.kt_total, splits));
+  p.a_mn = a_mn ? 1 : 0;
+  p.b_bytes = (bn * 128 + 1023) / 1024 * 1024;
+  p.stage_bytes = kABytes + p.b_bytes;
+  p.out = part;
+  p.ldo = n_cols;
+  p.out_bf16 = 0;
+  p.split_stride = m_rows * n_cols;
+  p.out_elems = static_cast<int64_t>(splits) * m_rows * n_cols;
+  dim3 grid(static_cast<unsigned>(ceil_div(n_cols, bn)), static_cast<unsigned>(ceil_div(m_rows, 128)),
+            static_cast<unsigned>(splits));
+  LevelTable unused{};
+  return launch_tc<B_TMA_K, 4>(ma, mb, ma, mb, p, unused, grid, s);
+}
+
+qlora_status splitk_reduce(const ReduceArgs& a, cudaStream_t s) {
+  const int64_t total = a.rows * a.cols;
+  const int grid = static_cast<int>(std::min<int64_t>(ceil_div(total, 256), 148 * 8));
+  count_launch();
+  splitk_reduce_kernel<<<grid, 256, 0, s>>>(
+      a.part, a.splits, a.rows, a.cols, a.pcols, a.lo, a.o1, a.ld1, a.trans1 ? 1 : 0, a.a1,
+      a.acc1 ? 1 : 0, static_cast<__nv_bfloat16*>(a.o2), a.ld2, a.a2, a.o2_lo,
+      static_cast<__nv_bfloat16*>(a.o3), a.ld3, a.a3, a.o3_lo);
+  return after_launch("splitk_reduce", s);
+}
+
+qlora_status transpose_to_bf16(const void* in, bool in_f32, int64_t rows, int cols, int64_t ld_in,
+                               void* out, int64_t ld_out, int lo_rows, cudaStream_t s) {
+  const int64_t total = rows * cols;
+  const int grid = static_cast<int>(std::min<int64_t>(ceil_div(total, 256), 148 * 8));
+  count_launch();
+  if (in_f32)
+    transpose_bf16_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float*>(in), rows, cols,
+                                                      ld_in, static_cast<__nv_bfloat16*>(out),
+                                                      ld_out, lo_rows);
+  else
+    transpose_bf16_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(in), rows, cols, ld_in,
+        static_cast<__nv_bfloat16*>(out), ld_out, lo_rows);
+  return after_launch("transpose_to_bf16", s);
+}
+
+}  // namespace qlora

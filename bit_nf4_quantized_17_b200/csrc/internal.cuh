@@ -40,6 +40,11 @@ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 // abi.cu: every kernel launch site calls this once per launch.
 void count_launch(unsigned n = 1);
 
+// abi.cu: status of the launch just enqueued.  With the environment variable
+// QLORA_SYNC_CHECK=1 the stream is synchronised after every launch and a
+// failing kernel is named on stderr (a debugging aid; off by default).
+qlora_status after_launch(const char* kernel, cudaStream_t s);
+
 inline bool aligned16(const void* p) {
   return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
 }

@@ -30,4 +30,53 @@ qlora_status simt_gemm(int kind_a, const Operand& a, int kind_b, const Operand& 
                        int64_t n, int64_t k, float alpha, const float* cin, void* c,
                        int64_t ldc, bool c_bf16, const LevelTable& t, cudaStream_t s);
 
+// gemm_tc.cu: tcgen05 / TMEM / TMA kernels.
+enum BMode { B_TMA_K = 0, B_DQ_K = 1, B_DQ_MN = 2 };
+
+// Columns of one half of a [hi | lo] LoRA operand buffer: r rounded up to 64.
+inline int32_t lora_span(int32_t r) { return (r + 63) / 64 * 64; }
+// Rows of one half of a transposed [hi ; lo] LoRA operand: r rounded up to 16.
+inline int32_t lora_rows(int32_t r) { return (r + 15) / 16 * 16; }
+
+int tc_split_count(int64_t m_tiles, int64_t k_tiles);
+
+// Y = X W^T + sU B^T, W dequantised on load; sU (M x 2*lora_span(r) bf16) holds
+// hi = bf16(s X A^T) in columns [0, r) and lo = bf16(s X A^T - hi) from column
+// lora_span(r), zero elsewhere.
+qlora_status tc_fused_forward(const QView& w, const LevelTable& t, const void* X, int64_t M,
+                              const void* sU, const void* B, int32_t r, void* Y,
+                              DeviceStatus* st, cudaStream_t s);
+// dX = dY W + sV A, W dequantised on load; sV laid out like sU, for s dY B.
+qlora_status tc_fused_dgrad(const QView& w, const LevelTable& t, const void* dY, int64_t M,
+                            const void* sV, const void* A, int32_t r, void* dX,
+                            DeviceStatus* st, cudaStream_t s);
+// part[z] (m_rows x n_cols fp32) = A . B^T over split z of the contraction; B has
+// b_rows rows, read as n_cols (rows past b_rows are zero).
+qlora_status tc_lora_gemm(const void* A, bool a_mn, int64_t m_rows, int64_t kdim, int64_t ld_a,
+                          const void* B, int64_t ld_b, int32_t b_rows, int32_t n_cols,
+                          float* part, int splits, DeviceStatus* st, cudaStream_t s);
+
+struct ReduceArgs {
+  const float* part;
+  int splits;
+  int64_t rows;
+  int cols, pcols, lo;
+  float* o1;
+  int64_t ld1;
+  bool trans1;
+  float a1;
+  bool acc1;
+  void* o2;
+  int64_t ld2;
+  float a2;
+  int o2_lo;
+  void* o3;
+  int64_t ld3;
+  float a3;
+  int o3_lo;
+};
+qlora_status splitk_reduce(const ReduceArgs& a, cudaStream_t s);
+qlora_status transpose_to_bf16(const void* in, bool in_f32, int64_t rows, int cols, int64_t ld_in,
+                               void* out, int64_t ld_out, int lo_rows, cudaStream_t s);
+
 }  // namespace qlora

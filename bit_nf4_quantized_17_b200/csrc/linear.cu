@@ -4,6 +4,17 @@
 // 到精通", 3(2)):   U = X A^T,  Y = X W^T + s U B^T,  s = alpha / r.
 // Backward (same pages, 6 and 3(3)): V = dY B, dX = dY W + s V A,
 // dB = s dY^T U, dA = s V^T X; no gradient for W.
+//
+// Tensor-core path (tcgen05, gemm_tc.cu), taken when M > 16, d_out % 8 == 0
+// and r % 8 == 0 (TMA needs 16-byte row strides):
+//   forward   U-GEMM (split-K) -> reduce (U fp32, sU bf16) -> fused
+//             dequant GEMM with the LoRA term as extra K stages          3 launches
+//   backward  U^T (transpose of the given U, or U-GEMM + reduce), B^T,
+//             V-GEMM -> reduce (sV, V^T), fused dequant dX GEMM,
+//             dB-GEMM -> reduce, dA-GEMM -> reduce                      8-9 launches
+// Other shapes take the CUDA-core contraction of gemm_simt.cu.
+#include <algorithm>
+
 #include "kernels.cuh"
 #include "linear.cuh"
 
@@ -19,37 +30,128 @@ QView view_of(const qlora_nf4& W) {
 
 float lora_scale(float alpha, int32_t r) { return alpha / static_cast<float>(r); }
 
+bool use_tc(int64_t M, int64_t N, int64_t K, int32_t r) {
+  (void)K;
+  return M > 16 && M < (int64_t(1) << 30) && N % 8 == 0 && r % 8 == 0;
+}
+
+int64_t pad8(int64_t v) { return (v + 7) / 8 * 8; }
+
+struct TcSplits {
+  int u, v, db, da;
+};
+
+TcSplits tc_splits(int64_t M, int64_t N, int64_t K) {
+  TcSplits s;
+  s.u = tc_split_count(ceil_div(M, 128), K / 64);
+  s.v = tc_split_count(ceil_div(M, 128), ceil_div(N, 64));
+  s.db = tc_split_count(ceil_div(N, 128), ceil_div(M, 64));
+  s.da = tc_split_count(ceil_div(K, 128), ceil_div(M, 64));
+  return s;
+}
+
+// Workspace regions of the tensor-core path (byte offsets; the status word is first).
+//   forward   sU [hi | lo] (M x 2*span bf16) | split-K partials
+//   backward  U^T [hi ; lo] (2*r16 x M8 bf16) | B^T (r x N bf16) | sV [hi | lo] |
+//             V^T [hi ; lo] | split-K partials
+struct TcLayout {
+  size_t su, part_f, ut, bt, sv, vt, part_b, fwd_end, bwd_end;
+};
+
+TcLayout tc_layout(int64_t M, int64_t N, int64_t K, int32_t r) {
+  const TcSplits sp = tc_splits(M, N, K);
+  const int64_t r16 = lora_rows(r), span = lora_span(r), mp = pad8(M);
+  TcLayout L{};
+  L.su = kStatusBytes;
+  L.part_f = L.su + align256(2 * M * 2 * span);
+  L.fwd_end = L.part_f + align256(sizeof(float) * sp.u * M * r16);
+  L.ut = kStatusBytes;
+  L.bt = L.ut + align256(2 * 2 * r16 * mp);
+  L.sv = L.bt + align256(2 * r * N);
+  L.vt = L.sv + align256(2 * M * 2 * span);
+  L.part_b = L.vt + align256(2 * 2 * r16 * mp);
+  const int64_t part = std::max(std::max(sp.u * M * r16, sp.v * M * r16),
+                                std::max(sp.db * N * 2 * r16, sp.da * K * 2 * r16));
+  L.bwd_end = L.part_b + align256(sizeof(float) * part);
+  return L;
+}
+
+ReduceArgs reduce_args(const float* part, int splits, int64_t rows, int cols, int pcols) {
+  ReduceArgs a{};
+  a.part = part;
+  a.splits = splits;
+  a.rows = rows;
+  a.cols = cols;
+  a.pcols = pcols;
+  return a;
+}
+
 }  // namespace
 
 LinearPlan plan_linear(int64_t M, int64_t N, int64_t K, int32_t r) {
   LinearPlan p;
+  if (use_tc(M, N, K, r)) {
+    TcLayout L = tc_layout(M, N, K, r);
+    p.fwd_workspace = L.fwd_end;
+    p.bwd_workspace = L.bwd_end;
+    return p;
+  }
   const size_t mr = align256(sizeof(float) * M * r);
   p.fwd_workspace = kStatusBytes + mr + align256(sizeof(float) * M * N);
   p.bwd_workspace = kStatusBytes + 2 * mr + align256(sizeof(float) * M * K);
   return p;
 }
 
+#define QLORA_TRY(x)                      \
+  do {                                    \
+    qlora_status _st = (x);               \
+    if (_st != QLORA_OK) return _st;      \
+  } while (0)
+
 qlora_status linear_forward(const qlora_nf4& W, const LevelTable& t, const void* A,
                             const void* B, int32_t r, float alpha, const void* X, int64_t M,
                             void* Y, float* U_save, void* workspace, cudaStream_t s) {
   const int64_t N = W.rows, K = W.cols;
-  char* ws = static_cast<char*>(workspace) + kStatusBytes;
-  float* u = U_save ? U_save : reinterpret_cast<float*>(ws);
-  ws += align256(sizeof(float) * M * r);
-  float* y0 = reinterpret_cast<float*>(ws);
   const QView w = view_of(W);
-  qlora_status st;
+  char* ws = static_cast<char*>(workspace);
+  auto* st = reinterpret_cast<DeviceStatus*>(ws);
+  const float sc = lora_scale(alpha, r);
+  if (use_tc(M, N, K, r)) {
+    const TcLayout L = tc_layout(M, N, K, r);
+    const TcSplits sp = tc_splits(M, N, K);
+    const int32_t r16 = lora_rows(r), span = lora_span(r);
+    char* su = ws + L.su;
+    float* part = reinterpret_cast<float*>(ws + L.part_f);
+    // the padding columns of [hi | lo] meet zero B columns in the MMA: keep them zero
+    if (cudaMemsetAsync(su, 0, sizeof(__nv_bfloat16) * M * 2 * span, s) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+    // U = X A^T (split-K over d_in) -> U_save (fp32) and sU = s U as bf16 hi + lo
+    QLORA_TRY(tc_lora_gemm(X, false, M, K, K, A, K, r, r16, part, sp.u, st, s));
+    ReduceArgs ra = reduce_args(part, sp.u, M, r, r16);
+    ra.o1 = U_save;
+    ra.ld1 = r;
+    ra.a1 = 1.0f;
+    ra.o2 = su;
+    ra.ld2 = 2 * span;
+    ra.a2 = sc;
+    ra.o2_lo = span;
+    QLORA_TRY(splitk_reduce(ra, s));
+    // Y = X W^T + sU B^T in one kernel
+    return tc_fused_forward(w, t, X, M, su, B, r, Y, st, s);
+  }
+  char* p = ws + kStatusBytes;
+  float* u = U_save ? U_save : reinterpret_cast<float*>(p);
+  p += align256(sizeof(float) * M * r);
+  float* y0 = reinterpret_cast<float*>(p);
   // U = X A^T
-  st = simt_gemm(OP_BF16_K, dense(X, K), OP_BF16_K, dense(A, K), M, r, K, 1.0f, nullptr, u, r,
-                 false, t, s);
-  if (st != QLORA_OK) return st;
+  QLORA_TRY(simt_gemm(OP_BF16_K, dense(X, K), OP_BF16_K, dense(A, K), M, r, K, 1.0f, nullptr, u,
+                      r, false, t, s));
   // Y0 = X W^T (W dequantised on the fly)
-  st = simt_gemm(OP_BF16_K, dense(X, K), OP_NF4_K, quantised(w), M, N, K, 1.0f, nullptr, y0, N,
-                 false, t, s);
-  if (st != QLORA_OK) return st;
+  QLORA_TRY(simt_gemm(OP_BF16_K, dense(X, K), OP_NF4_K, quantised(w), M, N, K, 1.0f, nullptr, y0,
+                      N, false, t, s));
   // Y = bf16(Y0 + s U B^T)
-  return simt_gemm(OP_F32_K, dense(u, r), OP_BF16_K, dense(B, r), M, N, r, lora_scale(alpha, r),
-                   y0, Y, N, true, t, s);
+  return simt_gemm(OP_F32_K, dense(u, r), OP_BF16_K, dense(B, r), M, N, r, sc, y0, Y, N, true, t,
+                   s);
 }
 
 qlora_status linear_backward(const qlora_nf4& W, const LevelTable& t, const void* A,
@@ -58,38 +160,98 @@ qlora_status linear_backward(const qlora_nf4& W, const LevelTable& t, const void
                              float* dB, bool accumulate, void* workspace, cudaStream_t s) {
   const int64_t N = W.rows, K = W.cols;
   const float sc = lora_scale(alpha, r);
-  char* ws = static_cast<char*>(workspace) + kStatusBytes;
-  float* u = reinterpret_cast<float*>(ws);
-  ws += align256(sizeof(float) * M * r);
-  float* v = reinterpret_cast<float*>(ws);
-  ws += align256(sizeof(float) * M * r);
-  float* dx0 = reinterpret_cast<float*>(ws);
   const QView w = view_of(W);
-  qlora_status st;
+  char* ws = static_cast<char*>(workspace);
+  auto* st = reinterpret_cast<DeviceStatus*>(ws);
+  if (use_tc(M, N, K, r)) {
+    const TcLayout L = tc_layout(M, N, K, r);
+    const TcSplits sp = tc_splits(M, N, K);
+    const int64_t mp = pad8(M);
+    const int32_t r16 = lora_rows(r), span = lora_span(r);
+    char* ut = ws + L.ut;
+    char* bt = ws + L.bt;
+    char* sv = ws + L.sv;
+    char* vt = ws + L.vt;
+    float* part = reinterpret_cast<float*>(ws + L.part_b);
+    if (cudaMemsetAsync(sv, 0, sizeof(__nv_bfloat16) * M * 2 * span, s) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+    // U^T as bf16 hi (rows [0, r)) + lo (rows [r16, r16 + r)), from the saved U or X A^T
+    if (U) {
+      QLORA_TRY(transpose_to_bf16(U, true, M, r, r, ut, mp, r16, s));
+    } else {
+      QLORA_TRY(tc_lora_gemm(X, false, M, K, K, A, K, r, r16, part, sp.u, st, s));
+      ReduceArgs ra = reduce_args(part, sp.u, M, r, r16);
+      ra.o3 = ut;
+      ra.ld3 = mp;
+      ra.a3 = 1.0f;
+      ra.o3_lo = r16;
+      QLORA_TRY(splitk_reduce(ra, s));
+    }
+    // B^T (r x N) so that V = dY B contracts two K-major operands
+    QLORA_TRY(transpose_to_bf16(B, false, N, r, r, bt, N, 0, s));
+    // V = dY B -> sV = s V as [hi | lo] and V^T as [hi ; lo]
+    QLORA_TRY(tc_lora_gemm(dY, false, M, N, N, bt, N, r, r16, part, sp.v, st, s));
+    {
+      ReduceArgs ra = reduce_args(part, sp.v, M, r, r16);
+      ra.o2 = sv;
+      ra.ld2 = 2 * span;
+      ra.a2 = sc;
+      ra.o2_lo = span;
+      ra.o3 = vt;
+      ra.ld3 = mp;
+      ra.a3 = 1.0f;
+      ra.o3_lo = r16;
+      QLORA_TRY(splitk_reduce(ra, s));
+    }
+    // dX = dY W + sV A in one kernel
+    if (dX) QLORA_TRY(tc_fused_dgrad(w, t, dY, M, sv, A, r, dX, st, s));
+    // dB = s dY^T U: rows d_out, contraction over tokens, hi and lo columns summed
+    QLORA_TRY(tc_lora_gemm(dY, true, N, M, N, ut, mp, 2 * r16, 2 * r16, part, sp.db, st, s));
+    {
+      ReduceArgs ra = reduce_args(part, sp.db, N, r, 2 * r16);
+      ra.lo = r16;
+      ra.o1 = dB;
+      ra.ld1 = r;
+      ra.a1 = sc;
+      ra.acc1 = accumulate;
+      QLORA_TRY(splitk_reduce(ra, s));
+    }
+    // dA = s V^T X: rows d_in, stored transposed as r x d_in
+    QLORA_TRY(tc_lora_gemm(X, true, K, M, K, vt, mp, 2 * r16, 2 * r16, part, sp.da, st, s));
+    ReduceArgs ra = reduce_args(part, sp.da, K, r, 2 * r16);
+    ra.lo = r16;
+    ra.o1 = dA;
+    ra.ld1 = K;
+    ra.trans1 = true;
+    ra.a1 = sc;
+    ra.acc1 = accumulate;
+    return splitk_reduce(ra, s);
+  }
+  char* p = ws + kStatusBytes;
+  float* u = reinterpret_cast<float*>(p);
+  p += align256(sizeof(float) * M * r);
+  float* v = reinterpret_cast<float*>(p);
+  p += align256(sizeof(float) * M * r);
+  float* dx0 = reinterpret_cast<float*>(p);
   if (!U) {
-    st = simt_gemm(OP_BF16_K, dense(X, K), OP_BF16_K, dense(A, K), M, r, K, 1.0f, nullptr, u, r,
-                   false, t, s);
-    if (st != QLORA_OK) return st;
+    QLORA_TRY(simt_gemm(OP_BF16_K, dense(X, K), OP_BF16_K, dense(A, K), M, r, K, 1.0f, nullptr, u,
+                        r, false, t, s));
     U = u;
   }
   // V = dY B      (B is N x r: element (j, n) = B[n][j])
-  st = simt_gemm(OP_BF16_K, dense(dY, N), OP_BF16_MN, dense(B, r), M, r, N, 1.0f, nullptr, v, r,
-                 false, t, s);
-  if (st != QLORA_OK) return st;
+  QLORA_TRY(simt_gemm(OP_BF16_K, dense(dY, N), OP_BF16_MN, dense(B, r), M, r, N, 1.0f, nullptr, v,
+                      r, false, t, s));
   if (dX) {
     // dX0 = dY W    (element (k, n) of the second operand = W[n][k])
-    st = simt_gemm(OP_BF16_K, dense(dY, N), OP_NF4_MN, quantised(w), M, K, N, 1.0f, nullptr,
-                   dx0, K, false, t, s);
-    if (st != QLORA_OK) return st;
+    QLORA_TRY(simt_gemm(OP_BF16_K, dense(dY, N), OP_NF4_MN, quantised(w), M, K, N, 1.0f, nullptr,
+                        dx0, K, false, t, s));
     // dX = bf16(dX0 + s V A)   (A is r x K: element (k, j) = A[j][k])
-    st = simt_gemm(OP_F32_K, dense(v, r), OP_BF16_MN, dense(A, K), M, K, r, sc, dx0, dX, K,
-                   true, t, s);
-    if (st != QLORA_OK) return st;
+    QLORA_TRY(simt_gemm(OP_F32_K, dense(v, r), OP_BF16_MN, dense(A, K), M, K, r, sc, dx0, dX, K,
+                        true, t, s));
   }
   // dB = s dY^T U (+ dB)   element (n, m) of dY^T = dY[m][n]; element (j, m) of U^T = U[m][j]
-  st = simt_gemm(OP_BF16_MN, dense(dY, N), OP_F32_MN, dense(U, r), N, r, M, sc,
-                 accumulate ? dB : nullptr, dB, r, false, t, s);
-  if (st != QLORA_OK) return st;
+  QLORA_TRY(simt_gemm(OP_BF16_MN, dense(dY, N), OP_F32_MN, dense(U, r), N, r, M, sc,
+                      accumulate ? dB : nullptr, dB, r, false, t, s));
   // dA = s V^T X (+ dA)
   return simt_gemm(OP_F32_MN, dense(v, r), OP_BF16_MN, dense(X, K), r, K, M, sc,
                    accumulate ? dA : nullptr, dA, K, false, t, s);

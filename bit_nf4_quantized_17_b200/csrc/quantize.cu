@@ -271,14 +271,15 @@ qlora_status launch_quantize(const void* W, int32_t w_dtype, const qlora_nf4& q,
   else
     launch_blocks(q.blocksize, static_cast<const __nv_bfloat16*>(W), n, t, q.codes, absmax, gmax,
                   st, s);
-  if (cudaPeekAtLastError() != cudaSuccess) return QLORA_ERR_CUDA;
+  if (after_launch("quantize_blocks", s) != QLORA_OK) return QLORA_ERR_CUDA;
   if (q.dq_blocksize) {
     count_launch(2);
     scale_sum_kernel<<<grid_for(nb, 256, 148 * 8), 256, 0, s>>>(absmax, nb, gmax, sum);
+    if (after_launch("scale_sum", s) != QLORA_OK) return QLORA_ERR_CUDA;
     const int64_t ng = ceil_div(nb, q.dq_blocksize);
     dq_groups_kernel<<<static_cast<unsigned>(ng), q.dq_blocksize, 0, s>>>(
         absmax, nb, gmax, sum, q.scale_codes, q.factors, q.mean);
-    if (cudaPeekAtLastError() != cudaSuccess) return QLORA_ERR_CUDA;
+    if (after_launch("dq_groups", s) != QLORA_OK) return QLORA_ERR_CUDA;
   }
   return QLORA_OK;
 }
@@ -296,7 +297,7 @@ qlora_status launch_dequantize(const qlora_nf4& q, const LevelTable& t, void* ou
   else
     dequantize_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(w, bs_shift, t,
                                                           static_cast<__nv_bfloat16*>(out));
-  return cudaPeekAtLastError() == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  return after_launch("dequantize", s);
 }
 
 }  // namespace qlora

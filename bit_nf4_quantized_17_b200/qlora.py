@@ -190,8 +190,10 @@ def qlora_dequantize(q, dtype=torch.float32, out=None, stream=None):
     return out
 
 
-def qlora_linear_fwd(q, A, B, alpha, X, Y=None, U_save=None, workspace=None, stream=None):
-    """Y = X W^T + (alpha/r) (X A^T) B^T.  Returns Y (and fills U_save if given)."""
+def qlora_linear_fwd(q, A, B, alpha, X, Y=None, U_save=None, workspace=None, stream=None,
+                     check=False):
+    """Y = X W^T + (alpha/r) (X A^T) B^T.  Returns Y (and fills U_save if given).
+    check=True synchronises and raises on a device-side error status."""
     M = X.shape[0]
     r = A.shape[0]
     if Y is None:
@@ -202,12 +204,15 @@ def qlora_linear_fwd(q, A, B, alpha, X, Y=None, U_save=None, workspace=None, str
     _ok(lib().qlora_linear_fwd(ctypes.byref(st), _ptr(A), _ptr(B), r, float(alpha), _ptr(X), M,
                                _ptr(Y), _ptr(U_save), _ptr(workspace), workspace.numel(),
                                _stream(stream)), "qlora_linear_fwd")
+    if check:
+        qlora_check(workspace, stream)
     return Y
 
 
 def qlora_linear_bwd(q, A, B, alpha, X, U, dY, dX=None, dA=None, dB=None, accumulate=False,
-                     want_dx=True, workspace=None, stream=None):
-    """Returns (dX, dA, dB); W gets no gradient."""
+                     want_dx=True, workspace=None, stream=None, check=False):
+    """Returns (dX, dA, dB); W gets no gradient.
+    check=True synchronises and raises on a device-side error status."""
     M = X.shape[0]
     r = A.shape[0]
     dev = X.device
@@ -224,6 +229,8 @@ def qlora_linear_bwd(q, A, B, alpha, X, U, dY, dX=None, dA=None, dB=None, accumu
                                _ptr(U), _ptr(dY), M, _ptr(dX) if want_dx else None, _ptr(dA),
                                _ptr(dB), 1 if accumulate else 0, _ptr(workspace),
                                workspace.numel(), _stream(stream)), "qlora_linear_bwd")
+    if check:
+        qlora_check(workspace, stream)
     return dX, dA, dB
 
 

@@ -16,7 +16,9 @@ What it computes, and where the method is stated:
   backward pass dX, dA, dB with no gradient for W ("LoRA 与 QLoRA：把大模型
   微调拆成可负担的工程", section 2 and section 6; "QLoRA技术从入门到精通",
   section 3(2) and 3(3)).
-* ``bf16.py``  - the bf16 <-> fp32 conversions the comparisons need.
+* ``bf16.py``  - the bf16 <-> fp32 conversions; the products use the
+  dequantised weight rounded to bf16 (``compute_weight``), the compute dtype
+  the pages name.
 
 Precision: the encoding steps are carried out in IEEE fp32 exactly as stated
 in each function (numpy float32 arithmetic rounds to nearest even); the linear
@@ -43,6 +45,7 @@ from .nf4 import (
     block_scales,
     quantize,
     dequantize,
+    compute_weight,
     storage_bits,
 )
 from .linear import lora_scale, linear_fwd, linear_bwd
@@ -51,6 +54,6 @@ __all__ = [
     "bf16_bits_to_f32", "f32_to_bf16_bits", "round_to_bf16",
     "nf4_levels", "nf4_raw_quantiles", "uniform_levels", "nearest_level",
     "block_absmax", "pack_nibbles", "unpack_nibbles", "fixed_point_mean",
-    "double_quantize", "dequantize_scales", "block_scales", "quantize", "dequantize",
+    "double_quantize", "dequantize_scales", "block_scales", "quantize", "dequantize", "compute_weight",
     "storage_bits", "lora_scale", "linear_fwd", "linear_bwd",
 ]

@@ -45,6 +45,8 @@ import math
 
 import numpy as np
 
+from .bf16 import round_to_bf16
+
 F32 = np.float32
 F64 = np.float64
 
@@ -260,6 +262,18 @@ def dequantize(qt):
     idx = unpack_nibbles(qt["codes"], n)
     sh = np.repeat(block_scales(qt), qt["blocksize"])[:n]
     return (qt["levels"][idx] * sh).astype(F32)
+
+
+def compute_weight(qt):
+    """The weight the products use: the dequantised weight rounded to bf16.
+
+    The pages restore the 4-bit weights to bf16 (or fp16) right before the
+    matrix product and drop them afterwards ("QLoRA技术从入门到精通", 3(2)
+    前向传播, 按需解压; "LoRA 与 QLoRA：用一块 GPU 微调大模型", 量化 part
+    "存储和计算"), with bf16 as the compute dtype ("LoRA 与 QLoRA：把大模型微调
+    拆成可负担的工程", 8).  Flattened, like ``dequantize``.
+    """
+    return round_to_bf16(dequantize(qt))
 
 
 def storage_bits(n, blocksize=64, dq_blocksize=256):

@@ -2,8 +2,9 @@
 
 Forward Y = X W^T + s (X A^T) B^T and backward dX = dY W + s V A,
 dB = s dY^T U, dA = s V^T X (V = dY B), with W the oracle's own dequantised
-weight.  bf16 outputs within the stated tolerance (tests/parity.py); fp32
-U, dA, dB within the same tolerance.  At the full sizes the oracle checks
+weight rounded to bf16 (the compute dtype the pages name).  bf16 outputs
+within the stated tolerance (tests/parity.py); fp32 U, dA, dB within the same
+bar measured in their own scale.  At the full sizes the oracle checks
 sampled token rows of Y and dX and every element of U, dA and dB.
 """
 
@@ -14,7 +15,7 @@ import torch
 import oracle
 from bit_nf4_quantized_17_b200 import qlora as Q
 from bit_nf4_quantized_17_b200 import workloads as WL
-from parity import assert_close, f64
+from parity import assert_close, assert_close_scaled, f64
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -22,7 +23,7 @@ DEV = "cuda"
 
 def _w_hat(W_cpu):
     ref = oracle.quantize(W_cpu.float().numpy(), 64, 256)
-    return oracle.dequantize(ref).reshape(W_cpu.shape)
+    return oracle.compute_weight(ref).reshape(W_cpu.shape)
 
 
 def _run(inp, alpha, rows=None, w_hat=None, check=True):
@@ -33,8 +34,8 @@ def _run(inp, alpha, rows=None, w_hat=None, check=True):
     q = Q.qlora_quantize(W.to(DEV))
     Ad, Bd, Xd, dYd = (t.to(DEV) for t in (A, B, X, dY))
     U = torch.empty((M, r), dtype=torch.float32, device=DEV)
-    Y = Q.qlora_linear_fwd(q, Ad, Bd, alpha, Xd, U_save=U)
-    dX, dA, dB = Q.qlora_linear_bwd(q, Ad, Bd, alpha, Xd, U, dYd)
+    Y = Q.qlora_linear_fwd(q, Ad, Bd, alpha, Xd, U_save=U, check=True)
+    dX, dA, dB = Q.qlora_linear_bwd(q, Ad, Bd, alpha, Xd, U, dYd, check=True)
     torch.cuda.synchronize()
     if not check:
         return q, Y, U, dX, dA, dB
@@ -44,13 +45,13 @@ def _run(inp, alpha, rows=None, w_hat=None, check=True):
     y_ref, _ = oracle.linear_fwd(w_hat, a, b, alpha, x[sel])
     assert_close(f64(Y)[sel], y_ref, "Y")
     u_ref = x @ a.T
-    assert_close(U, u_ref, "U")
+    assert_close_scaled(U, u_ref, "U")
     dx_ref, _, _ = oracle.linear_bwd(w_hat, a, b, alpha, x[sel], dy[sel])
     assert_close(f64(dX)[sel], dx_ref, "dX")
     s = oracle.lora_scale(alpha, r)
     v = dy @ b
-    assert_close(dA, s * (v.T @ x), "dA")
-    assert_close(dB, s * (dy.T @ u_ref), "dB")
+    assert_close_scaled(dA, s * (v.T @ x), "dA")
+    assert_close_scaled(dB, s * (dy.T @ u_ref), "dB")
     return q, Y, U, dX, dA, dB
 
 

@@ -61,3 +61,16 @@ def test_uniform_grid_points_printed_on_page(golden):
     assert q[0] == -1.0 and q[15] == 1.0
     assert q[int(g["index_0"][0])] == np.float32(float(g["level_0"][0]))
     np.testing.assert_allclose(np.diff(q.astype(np.float64)), 2.0 / 15.0, rtol=1e-6)
+
+
+def test_bf16_rounding_matches_library_conversion():
+    import torch
+    rng = np.random.default_rng(11)
+    x = np.concatenate([rng.standard_normal(20000).astype(np.float32) * 10.0 ** rng.integers(-6, 6, 20000),
+                        np.array([1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -(1.0 + 2 ** -8), 0.0, -0.0,
+                                  3.4e38, 1e-40], np.float32)]).astype(np.float32)
+    ref = torch.from_numpy(x).bfloat16().view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(oracle.f32_to_bf16_bits(x), ref)
+    # ties go to even: 1 + 2^-8 is halfway between 1 and 1 + 2^-7
+    assert oracle.round_to_bf16(np.float32(1.0 + 2 ** -8)) == np.float32(1.0)
+    assert oracle.round_to_bf16(np.float32(1.0 + 3 * 2 ** -8)) == np.float32(1.0 + 2 ** -6)
