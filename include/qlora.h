@@ -117,6 +117,23 @@ qlora_status qlora_nf4_sizes(int64_t rows, int64_t cols, int32_t blocksize,
 qlora_status qlora_quantize(const void* W, int32_t w_dtype, const qlora_nf4* q,
                             void* workspace, size_t workspace_bytes, void* stream);
 
+/* qlora_quantize without a workspace argument, for callers that cannot
+ * allocate one: code whose device memory belongs to a pool that has already
+ * reserved the GPU, and loops that cannot pay the device-wide synchronisation
+ * of cudaMalloc/cudaFree.  The pages have no counterpart to this call; it is a
+ * library convenience.  Same inputs, outputs and results as qlora_quantize.
+ * The reduction workspace is a fixed array in the library's own device memory
+ * (one copy per GPU that loads the library, 4 MiB + 512 B, kept until exit):
+ * at most 2^20 blocks (64 Mi weights at blocksize 64), larger tensors return
+ * QLORA_ERR_WORKSPACE.  All calls on a device share the array: calls whose
+ * work overlaps on the GPU race; calls on one stream are safe.  status_out
+ * (device, 4 bytes, may be NULL) receives the device status when the work
+ * completes: 0, or QLORA_ERR_NONFINITE for a NaN or infinite weight.  The
+ * first call on a device looks up the array (cudaGetSymbolAddress on the
+ * current device); make that first call before any stream capture. */
+qlora_status qlora_quantize_noalloc(const void* W, int32_t w_dtype, const qlora_nf4* q,
+                                    uint32_t* status_out, void* stream);
+
 /* Dequantise *q into W_out (device, rows*cols values of out_dtype):
  * fp32 out is w = fp32(level[idx] * s_b) bit for bit; bf16 out is that value
  * rounded to nearest even.  Needs no workspace. */
