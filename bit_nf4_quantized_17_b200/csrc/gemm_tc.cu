@@ -137,11 +137,13 @@ __device__ __forceinline__ void store16(const TcArgs& p, int64_t row, int64_t co
   }
 }
 
-template <int BMODE, int STAGES>
+template <int BMODE, int STAGES, int MT>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
                const TcArgs p, const LevelTable tab) {
+  // MT accumulators of 128 rows share every B tile: a CTA covers 128*MT rows.
+  constexpr int kA = kABytes * MT;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -153,7 +155,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.y * 128;
+  const int m0 = blockIdx.y * 128 * MT;
   const int n0 = blockIdx.x * p.bn;
   const int kt0 = blockIdx.z * p.k_tiles;
   const int k_tiles = min(p.k_tiles, p.kt_total - kt0);
@@ -192,35 +194,41 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const uint32_t ph = (kt / STAGES) & 1;
       if (!ptx::mbar_wait(&empty[s], ph ^ 1, kTimeoutCycles, abort_flag)) break;
       uint8_t* sa = smem + s * p.stage_bytes;
-      uint8_t* sb = sa + kABytes;
+      uint8_t* sb = sa + kA;
       uint8_t* sc = sb + p.b_bytes;
       if (kt < k_tiles) {
         const int kg = kt0 + kt;
-        const uint32_t bytes = kABytes + (BMODE == B_TMA_K ? p.bn * 128 : kCodeBytes);
+        const uint32_t bytes = kA + (BMODE == B_TMA_K ? p.bn * 128 : kCodeBytes);
         ptx::mbar_arrive_expect_tx(&full_tma[s], bytes);
         if (p.a_mn) {
+          // MN-major A (only with MT == 1): two 64-row halves
           ptx::tma_load_2d(&tmA, &full_tma[s], sa, m0, kg * 64);
           ptx::tma_load_2d(&tmA, &full_tma[s], sa + 8192, m0 + 64, kg * 64);
         } else {
           ptx::tma_load_2d(&tmA, &full_tma[s], sa, kg * 64, m0);
         }
-        if (BMODE == B_TMA_K)
+        if (BMODE == B_TMA_K) {
           ptx::tma_load_2d(&tmB, &full_tma[s], sb, kg * 64, n0);
-        else if (BMODE == B_DQ_K)
+        } else if (BMODE == B_DQ_K) {
           ptx::tma_load_2d(&tmB, &full_tma[s], sc, kg * 32, n0);
-        else
-          ptx::tma_load_2d(&tmB, &full_tma[s], sc, n0 / 2, kg * 64);
+        } else {
+          // four 32-byte column slices (one 64-weight block each) of 64 W rows
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            ptx::tma_load_2d(&tmB, &full_tma[s], sc + q * 2048, n0 / 2 + 32 * q, kg * 64);
+        }
       } else {
         // extension stage tt: A2 columns [64 tt, 64 tt + 64) of [hi | lo], B2 ranks
         // [64 (tt mod half), ...): both halves multiply the same B2 tiles
         const int tt = kt - k_tiles;
         const int k2a = tt * 64;
         const int k2b = (tt % p.k2_half) * 64;
-        ptx::mbar_arrive_expect_tx(&full_tma[s], kABytes + 32768);
+        ptx::mbar_arrive_expect_tx(&full_tma[s], kA + 32768);
         ptx::tma_load_2d(&tmA2, &full_tma[s], sa, k2a, m0);
         if (p.b2_mn) {
 #pragma unroll
-          for (int h = 0; h < 4; ++h) ptx::tma_load_2d(&tmB2, &full_tma[s], sb + h * 8192, n0 + 64 * h, k2b);
+          for (int h = 0; h < 4; ++h)
+            ptx::tma_load_2d(&tmB2, &full_tma[s], sb + h * 8192, n0 + 64 * h, k2b);
         } else {
           ptx::tma_load_2d(&tmB2, &full_tma[s], sb, k2b, n0);
         }
@@ -243,16 +251,19 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         break;
       ptx::tc_fence_after();
       const uint32_t a_addr = ptx::smem_u32(smem + s * p.stage_bytes);
-      const uint32_t b_addr = a_addr + kABytes;
+      const uint32_t b_addr = a_addr + kA;
       const bool a_mn = !ext && p.a_mn;
       const bool b_mn = ext ? (p.b2_mn != 0) : (BMODE == B_DQ_MN);
       const int steps = (ext && ((kt - k_tiles) % p.k2_half) == p.k2_half - 1) ? p.k2_last_steps : 4;
       for (int ks = 0; ks < steps; ++ks) {
-        const uint64_t ad = a_mn ? ptx::sw128_desc(a_addr + ks * 2048, 8192, 1024)
-                                 : ptx::sw128_desc(a_addr + ks * 32, 16, 1024);
         const uint64_t bd = b_mn ? ptx::sw128_desc(b_addr + ks * 2048, 8192, 1024)
                                  : ptx::sw128_desc(b_addr + ks * 32, 16, 1024);
-        ptx::umma_bf16(tmem, ad, bd, ext ? idesc2 : idesc, (kt | ks) != 0 ? 1u : 0u);
+#pragma unroll
+        for (int t = 0; t < MT; ++t) {
+          const uint64_t ad = a_mn ? ptx::sw128_desc(a_addr + ks * 2048, 8192, 1024)
+                                   : ptx::sw128_desc(a_addr + t * kABytes + ks * 32, 16, 1024);
+          ptx::umma_bf16(tmem + t * p.bn, ad, bd, ext ? idesc2 : idesc, (kt | ks) != 0 ? 1u : 0u);
+        }
       }
       ptx::umma_commit(&empty[s]);
     }
@@ -262,68 +273,42 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     const int td = threadIdx.x - 128;
     if (BMODE != B_TMA_K) {
       // ---------------------------------------------------- dequantisation
+      // forward: thread td expands W row n0 + td (one 64-weight block per stage);
+      // backward: thread td expands block q = td / 64 of W row (stage rows) + td % 64.
       float lv[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) lv[j] = tab.level[j];
       const float mu = (p.w.dq_shift >= 0) ? __ldg(p.w.mean) : 0.0f;
-      int row, q;            // row of the codes tile, block within the row
-      int64_t wrow, kb;      // W row and 64-block column of this thread's block
-      if (BMODE == B_DQ_K) {
-        row = td;
-        q = 0;
-      } else {
-        row = td >> 2;
-        q = td & 3;
-      }
+      const int row = (BMODE == B_DQ_K) ? td : (td & 63);
+      const int q = (BMODE == B_DQ_K) ? 0 : (td >> 6);
       for (int kt = 0; kt < k_tiles; ++kt) {
         const int s = kt % STAGES;
         const uint32_t ph = (kt / STAGES) & 1;
         const int kg = kt0 + kt;
-        if (BMODE == B_DQ_K) {
-          wrow = n0 + row;
-          kb = kg;
-        } else {
-          wrow = static_cast<int64_t>(kg) * 64 + row;
-          kb = n0 / 64 + q;
-        }
+        const int64_t wrow = (BMODE == B_DQ_K) ? static_cast<int64_t>(n0) + row
+                                               : static_cast<int64_t>(kg) * 64 + row;
+        const int64_t kb = (BMODE == B_DQ_K) ? kg : (n0 / 64 + q);
         bool valid = wrow < p.w.rows && kb < p.kblocks;
         if (valid && (wrow * p.kblocks + kb >= p.nblocks)) {
           report(p.st, QLORA_ERR_SHAPE, 201u);
           valid = false;
         }
+        // rows or blocks outside W get a zero table, hence zero weights
         const float sc = valid ? block_scale(p.w, wrow * p.kblocks + kb, mu) : 0.0f;
         if (!ptx::mbar_wait(&full_tma[s], ph, kTimeoutCycles, abort_flag)) break;
         uint8_t* sa = smem + s * p.stage_bytes;
-        uint8_t* sb = sa + kABytes;
-        const uint8_t* sc_codes = sb + p.b_bytes;
-        const uint8_t* src = (BMODE == B_DQ_K) ? sc_codes + row * 32 : sc_codes + row * 128 + q * 32;
-        const int h0 = (BMODE == B_DQ_K) ? ((row >> 2) & 1) : (row & 1);
-        // the two 16-byte halves are read in an order that spreads banks
-        const uint4 first = *reinterpret_cast<const uint4*>(src + 16 * h0);
-        const uint4 second = *reinterpret_cast<const uint4*>(src + 16 * (h0 ^ 1));
-        uint4 cw[2];
-        cw[0] = h0 ? second : first;
-        cw[1] = h0 ? first : second;
+        uint8_t* sb = sa + kA;
+        const uint8_t* codes = sb + p.b_bytes;
+        const uint8_t* src = (BMODE == B_DQ_K) ? codes + row * 32 : codes + q * 2048 + row * 32;
+        const uint4 c0 = *reinterpret_cast<const uint4*>(src);
+        const uint4 c1 = *reinterpret_cast<const uint4*>(src + 16);
         uint32_t L[4], H[4];
         block_tables(lv, sc, L, H);
-        uint32_t words[8] = {cw[0].x, cw[0].y, cw[0].z, cw[0].w,
-                             cw[1].x, cw[1].y, cw[1].z, cw[1].w};
-        if (BMODE == B_DQ_MN) {
-          // threads of one row write different chunks at the same time (bank
-          // spread): word j of this thread becomes chunk (j + 2q) mod 8
-          uint32_t t8[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) t8[j] = (q & 1) ? words[(j + 2) & 7] : words[j];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) words[j] = (q & 2) ? t8[(j + 4) & 7] : t8[j];
-        }
+        const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
         uint8_t* dst_row = (BMODE == B_DQ_K) ? sb + row * 128 : sb + q * 8192 + row * 128;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int c = (BMODE == B_DQ_K) ? j : ((j + 2 * q) & 7);
-          const uint4 v = valid ? expand8(words[j], L, H) : make_uint4(0u, 0u, 0u, 0u);
-          *reinterpret_cast<uint4*>(dst_row + 16 * (c ^ (row & 7))) = v;
-        }
+        for (int j = 0; j < 8; ++j)
+          *reinterpret_cast<uint4*>(dst_row + 16 * (j ^ (row & 7))) = expand8(words[j], L, H);
         ptx::fence_proxy_async_smem();
         ptx::mbar_arrive(&full_b[s]);
       }
@@ -335,11 +320,15 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       ptx::tc_fence_after();
       const int quarter = warp & 3;
       const int group = (warp - 4) >> 2;
-      const int64_t row = static_cast<int64_t>(m0) + 32 * quarter + lane;
       const int nchunks = p.bn / 16;
-      for (int c = group; c < nchunks; c += 2) {
+      // MT == 2: group g drains accumulator g; MT == 1: the groups split the columns
+      const int t = (MT == 2) ? group : 0;
+      const int c_first = (MT == 2) ? 0 : group;
+      const int c_step = (MT == 2) ? 1 : 2;
+      const int64_t row = static_cast<int64_t>(m0) + 128 * t + 32 * quarter + lane;
+      for (int c = c_first; c < nchunks; c += c_step) {
         uint32_t r[16];
-        ptx::tmem_ld_x16(tmem + (static_cast<uint32_t>(32 * quarter) << 16) + c * 16, r);
+        ptx::tmem_ld_x16(tmem + (static_cast<uint32_t>(32 * quarter) << 16) + t * p.bn + c * 16, r);
         ptx::tmem_ld_wait();
         store16(p, row, static_cast<int64_t>(n0) + c * 16, r);
       }
@@ -460,21 +449,21 @@ int pow2_cols(int bn) {
   return c;
 }
 
-template <int BMODE, int STAGES>
+template <int BMODE, int STAGES, int MT>
 qlora_status launch_tc(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2,
                        const CUtensorMap& b2, TcArgs p, const LevelTable& t, dim3 grid,
                        cudaStream_t s) {
   const size_t smem = 1024 + static_cast<size_t>(STAGES) * p.stage_bytes + 256;
   static bool configured = false;
   if (!configured) {
-    if (cudaFuncSetAttribute(tc_gemm_kernel<BMODE, STAGES>,
+    if (cudaFuncSetAttribute(tc_gemm_kernel<BMODE, STAGES, MT>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(232448)) != cudaSuccess)
       return QLORA_ERR_CUDA;
     configured = true;
   }
   count_launch();
-  tc_gemm_kernel<BMODE, STAGES><<<grid, kThreads, smem, s>>>(a, b, a2, b2, p, t);
+  tc_gemm_kernel<BMODE, STAGES, MT><<<grid, kThreads, smem, s>>>(a, b, a2, b2, p, t);
   return after_launch(BMODE == B_TMA_K ? "tc_gemm(lora)" : BMODE == B_DQ_K ? "tc_gemm(fwd)" : "tc_gemm(dgrad)", s);
 }
 
@@ -507,9 +496,9 @@ qlora_status tc_fused_forward(const QView& w, const LevelTable& t, const void* X
                               DeviceStatus* st, cudaStream_t s) {
   const int64_t N = w.rows, K = w.cols;
   CUtensorMap ma, mb, ma2, mb2;
-  if (!make_map(&ma, X, true, K, M, K, 64, 128, true) ||
+  if (!make_map(&ma, X, true, K, M, K, 64, 256, true) ||
       !make_map(&mb, w.codes, false, K / 2, N, K / 2, 32, 256, false) ||
-      !make_map(&ma2, sU, true, 2 * lora_span(r), M, 2 * lora_span(r), 64, 128, true) ||
+      !make_map(&ma2, sU, true, 2 * lora_span(r), M, 2 * lora_span(r), 64, 256, true) ||
       !make_map(&mb2, B, true, r, N, r, 64, 256, true))
     return QLORA_ERR_CUDA;
   TcArgs p = base_args(static_cast<int>(M), static_cast<int>(N), 256, st);
@@ -518,7 +507,8 @@ qlora_status tc_fused_forward(const QView& w, const LevelTable& t, const void* X
   p.k2_tiles = 2 * p.k2_half;
   p.k2_last_steps = ((r - 64 * (p.k2_half - 1)) + 15) / 16;
   p.b_bytes = 32768;
-  p.stage_bytes = kABytes + 32768 + kCodeBytes;
+  p.stage_bytes = 2 * kABytes + 32768 + kCodeBytes;
+  p.tmem_cols = 512;
   p.w = w;
   p.kblocks = static_cast<int>(K / 64);
   p.out = Y;
@@ -526,8 +516,8 @@ qlora_status tc_fused_forward(const QView& w, const LevelTable& t, const void* X
   p.out_bf16 = 1;
   p.out_elems = M * N;
   p.nblocks = N * K / 64;
-  dim3 grid(static_cast<unsigned>(ceil_div(N, 256)), static_cast<unsigned>(ceil_div(M, 128)), 1);
-  return launch_tc<B_DQ_K, 3>(ma, mb, ma2, mb2, p, t, grid, s);
+  dim3 grid(static_cast<unsigned>(ceil_div(N, 256)), static_cast<unsigned>(ceil_div(M, 256)), 1);
+  return launch_tc<B_DQ_K, 3, 2>(ma, mb, ma2, mb2, p, t, grid, s);
 }
 
 qlora_status tc_fused_dgrad(const QView& w, const LevelTable& t, const void* dY, int64_t M,
@@ -535,9 +525,9 @@ qlora_status tc_fused_dgrad(const QView& w, const LevelTable& t, const void* dY,
                             DeviceStatus* st, cudaStream_t s) {
   const int64_t N = w.rows, K = w.cols;
   CUtensorMap ma, mb, ma2, mb2;
-  if (!make_map(&ma, dY, true, N, M, N, 64, 128, true) ||
-      !make_map(&mb, w.codes, false, K / 2, N, K / 2, 128, 64, false) ||
-      !make_map(&ma2, sV, true, 2 * lora_span(r), M, 2 * lora_span(r), 64, 128, true) ||
+  if (!make_map(&ma, dY, true, N, M, N, 64, 256, true) ||
+      !make_map(&mb, w.codes, false, K / 2, N, K / 2, 32, 64, false) ||
+      !make_map(&ma2, sV, true, 2 * lora_span(r), M, 2 * lora_span(r), 64, 256, true) ||
       !make_map(&mb2, A, true, K, r, K, 64, 64, true))
     return QLORA_ERR_CUDA;
   TcArgs p = base_args(static_cast<int>(M), static_cast<int>(K), 256, st);
@@ -547,7 +537,8 @@ qlora_status tc_fused_dgrad(const QView& w, const LevelTable& t, const void* dY,
   p.k2_last_steps = ((r - 64 * (p.k2_half - 1)) + 15) / 16;
   p.b2_mn = 1;
   p.b_bytes = 32768;
-  p.stage_bytes = kABytes + 32768 + kCodeBytes;
+  p.stage_bytes = 2 * kABytes + 32768 + kCodeBytes;
+  p.tmem_cols = 512;
   p.w = w;
   p.kblocks = static_cast<int>(K / 64);
   p.out = dX;
@@ -555,8 +546,8 @@ qlora_status tc_fused_dgrad(const QView& w, const LevelTable& t, const void* dY,
   p.out_bf16 = 1;
   p.out_elems = M * K;
   p.nblocks = N * K / 64;
-  dim3 grid(static_cast<unsigned>(ceil_div(K, 256)), static_cast<unsigned>(ceil_div(M, 128)), 1);
-  return launch_tc<B_DQ_MN, 3>(ma, mb, ma2, mb2, p, t, grid, s);
+  dim3 grid(static_cast<unsigned>(ceil_div(K, 256)), static_cast<unsigned>(ceil_div(M, 256)), 1);
+  return launch_tc<B_DQ_MN, 3, 2>(ma, mb, ma2, mb2, p, t, grid, s);
 }
 
 // part[z] (m_rows x n_cols fp32) = A . B^T over split z of the contraction; A is
@@ -585,7 +576,7 @@ qlora_status tc_lora_gemm(const void* A, bool a_mn, int64_t m_rows, int64_t kdim
   dim3 grid(static_cast<unsigned>(ceil_div(n_cols, bn)), static_cast<unsigned>(ceil_div(m_rows, 128)),
             static_cast<unsigned>(splits));
   LevelTable unused{};
-  return launch_tc<B_TMA_K, 4>(ma, mb, ma, mb, p, unused, grid, s);
+  return launch_tc<B_TMA_K, 4, 1>(ma, mb, ma, mb, p, unused, grid, s);
 }
 
 qlora_status splitk_reduce(const ReduceArgs& a, cudaStream_t s) {
