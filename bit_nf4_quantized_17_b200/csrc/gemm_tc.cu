@@ -36,7 +36,8 @@ namespace {
 
 constexpr int kThreads = 384;
 constexpr int kABytes = 16384;   // 128 rows x 64 bf16
-constexpr int kCodeBytes = 8192;  // 256 W rows x 32 B (fwd) or 64 W rows x 128 B (bwd)
+constexpr int kCodeBytes = 8192;  // codes of one stage: 256 W rows x 32 B (fwd) or 4 x 64 x 32 B (bwd)
+constexpr int kCodeStages = 4;    // depth of the codes ring
 constexpr long long kTimeoutCycles = 4000000000ll;  // ~2 s at 1.9 GHz
 
 struct TcArgs {
@@ -144,13 +145,18 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                const TcArgs p, const LevelTable tab) {
   // MT accumulators of 128 rows share every B tile: a CTA covers 128*MT rows.
   constexpr int kA = kABytes * MT;
+  constexpr bool kDq = BMODE != B_TMA_K;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint64_t* full_tma = reinterpret_cast<uint64_t*>(smem + STAGES * p.stage_bytes);
-  uint64_t* full_b = full_tma + STAGES;
+  // [STAGES x (A | B)] [kCodeStages x codes] [barriers]
+  uint8_t* codes_ring = smem + STAGES * p.stage_bytes;
+  uint64_t* full_a = reinterpret_cast<uint64_t*>(codes_ring + (kDq ? kCodeStages * kCodeBytes : 0));
+  uint64_t* full_b = full_a + STAGES;
   uint64_t* empty = full_b + STAGES;
-  uint64_t* accum = empty + STAGES;
+  uint64_t* codes_full = empty + STAGES;
+  uint64_t* codes_empty = codes_full + kCodeStages;
+  uint64_t* accum = codes_empty + kCodeStages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -163,9 +169,13 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      ptx::mbar_init(&full_tma[s], 1);
+      ptx::mbar_init(&full_a[s], 1);
       ptx::mbar_init(&full_b[s], 256);
       ptx::mbar_init(&empty[s], 1);
+    }
+    for (int s = 0; s < kCodeStages; ++s) {
+      ptx::mbar_init(&codes_full[s], 1);
+      ptx::mbar_init(&codes_empty[s], 256);
     }
     ptx::mbar_init(accum, 1);
     *abort_flag = 0;
@@ -188,56 +198,75 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------ TMA producer
-    int issued = 0;
-    for (int kt = 0; kt < total; ++kt) {
+    // A (and B when it is bf16) go into stage kt % STAGES once the MMAs of
+    // its previous use are done; the 4-bit codes run up to kCodeStages tiles
+    // ahead in their own ring, freed as soon as the dequant warps read them.
+    int issued = 0, kc = 0;
+    bool ok = true;
+    auto issue_codes = [&](int upto) {
+      while (ok && kc < k_tiles && kc < upto) {
+        const int cs = kc % kCodeStages;
+        if (!ptx::mbar_wait(&codes_empty[cs], ((kc / kCodeStages) & 1) ^ 1, kTimeoutCycles,
+                            abort_flag)) {
+          ok = false;
+          break;
+        }
+        uint8_t* dst = codes_ring + cs * kCodeBytes;
+        const int kg = kt0 + kc;
+        ptx::mbar_arrive_expect_tx(&codes_full[cs], kCodeBytes);
+        if (BMODE == B_DQ_K) {
+          ptx::tma_load_2d(&tmB, &codes_full[cs], dst, kg * 32, n0);
+        } else {
+          // four 32-byte column slices (one 64-weight block each) of 64 W rows
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            ptx::tma_load_2d(&tmB, &codes_full[cs], dst + q * 2048, n0 / 2 + 32 * q, kg * 64);
+        }
+        ++kc;
+      }
+    };
+    if (kDq) issue_codes(kCodeStages);
+    for (int kt = 0; kt < total && ok; ++kt) {
       const int s = kt % STAGES;
       const uint32_t ph = (kt / STAGES) & 1;
       if (!ptx::mbar_wait(&empty[s], ph ^ 1, kTimeoutCycles, abort_flag)) break;
       uint8_t* sa = smem + s * p.stage_bytes;
       uint8_t* sb = sa + kA;
-      uint8_t* sc = sb + p.b_bytes;
       if (kt < k_tiles) {
         const int kg = kt0 + kt;
-        const uint32_t bytes = kA + (BMODE == B_TMA_K ? p.bn * 128 : kCodeBytes);
-        ptx::mbar_arrive_expect_tx(&full_tma[s], bytes);
+        ptx::mbar_arrive_expect_tx(&full_a[s], kA + (kDq ? 0 : p.bn * 128));
         if (p.a_mn) {
           // MN-major A (only with MT == 1): two 64-row halves
-          ptx::tma_load_2d(&tmA, &full_tma[s], sa, m0, kg * 64);
-          ptx::tma_load_2d(&tmA, &full_tma[s], sa + 8192, m0 + 64, kg * 64);
+          ptx::tma_load_2d(&tmA, &full_a[s], sa, m0, kg * 64);
+          ptx::tma_load_2d(&tmA, &full_a[s], sa + 8192, m0 + 64, kg * 64);
         } else {
-          ptx::tma_load_2d(&tmA, &full_tma[s], sa, kg * 64, m0);
+          ptx::tma_load_2d(&tmA, &full_a[s], sa, kg * 64, m0);
         }
-        if (BMODE == B_TMA_K) {
-          ptx::tma_load_2d(&tmB, &full_tma[s], sb, kg * 64, n0);
-        } else if (BMODE == B_DQ_K) {
-          ptx::tma_load_2d(&tmB, &full_tma[s], sc, kg * 32, n0);
-        } else {
-          // four 32-byte column slices (one 64-weight block each) of 64 W rows
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            ptx::tma_load_2d(&tmB, &full_tma[s], sc + q * 2048, n0 / 2 + 32 * q, kg * 64);
-        }
+        if (!kDq) ptx::tma_load_2d(&tmB, &full_a[s], sb, kg * 64, n0);
       } else {
         // extension stage tt: A2 columns [64 tt, 64 tt + 64) of [hi | lo], B2 ranks
         // [64 (tt mod half), ...): both halves multiply the same B2 tiles
         const int tt = kt - k_tiles;
         const int k2a = tt * 64;
         const int k2b = (tt % p.k2_half) * 64;
-        ptx::mbar_arrive_expect_tx(&full_tma[s], kA + 32768);
-        ptx::tma_load_2d(&tmA2, &full_tma[s], sa, k2a, m0);
+        ptx::mbar_arrive_expect_tx(&full_a[s], kA + 32768);
+        ptx::tma_load_2d(&tmA2, &full_a[s], sa, k2a, m0);
         if (p.b2_mn) {
 #pragma unroll
           for (int h = 0; h < 4; ++h)
-            ptx::tma_load_2d(&tmB2, &full_tma[s], sb + h * 8192, n0 + 64 * h, k2b);
+            ptx::tma_load_2d(&tmB2, &full_a[s], sb + h * 8192, n0 + 64 * h, k2b);
         } else {
-          ptx::tma_load_2d(&tmB2, &full_tma[s], sb, k2b, n0);
+          ptx::tma_load_2d(&tmB2, &full_a[s], sb, k2b, n0);
         }
       }
       ++issued;
+      if (kDq) issue_codes(kt + 1 + kCodeStages);
     }
     // never leave with copies in flight into this CTA's shared memory
     for (int kt = max(0, issued - STAGES); kt < issued; ++kt)
-      ptx::mbar_wait(&full_tma[kt % STAGES], (kt / STAGES) & 1, kTimeoutCycles, nullptr);
+      ptx::mbar_wait(&full_a[kt % STAGES], (kt / STAGES) & 1, kTimeoutCycles, nullptr);
+    for (int c = max(0, kc - kCodeStages); c < kc; ++c)
+      ptx::mbar_wait(&codes_full[c % kCodeStages], (c / kCodeStages) & 1, kTimeoutCycles, nullptr);
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------ MMA issuer
     const uint32_t idesc = ptx::idesc_bf16(128, p.bn, p.a_mn, BMODE == B_DQ_MN ? 1 : 0);
@@ -245,10 +274,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     for (int kt = 0; kt < total; ++kt) {
       const int s = kt % STAGES;
       const uint32_t ph = (kt / STAGES) & 1;
-      if (!ptx::mbar_wait(&full_tma[s], ph, kTimeoutCycles, abort_flag)) break;
+      if (!ptx::mbar_wait(&full_a[s], ph, kTimeoutCycles, abort_flag)) break;
       const bool ext = kt >= k_tiles;
-      if (BMODE != B_TMA_K && !ext && !ptx::mbar_wait(&full_b[s], ph, kTimeoutCycles, abort_flag))
-        break;
+      if (kDq && !ext && !ptx::mbar_wait(&full_b[s], ph, kTimeoutCycles, abort_flag)) break;
       ptx::tc_fence_after();
       const uint32_t a_addr = ptx::smem_u32(smem + s * p.stage_bytes);
       const uint32_t b_addr = a_addr + kA;
@@ -271,7 +299,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     ptx::mbar_wait(accum, 0, kTimeoutCycles, nullptr);  // MMAs done before TMEM is freed
   } else if (warp >= 4) {
     const int td = threadIdx.x - 128;
-    if (BMODE != B_TMA_K) {
+    if (kDq) {
       // ---------------------------------------------------- dequantisation
       // forward: thread td expands W row n0 + td (one 64-weight block per stage);
       // backward: thread td expands block q = td / 64 of W row (stage rows) + td % 64.
@@ -281,30 +309,44 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const float mu = (p.w.dq_shift >= 0) ? __ldg(p.w.mean) : 0.0f;
       const int row = (BMODE == B_DQ_K) ? td : (td & 63);
       const int q = (BMODE == B_DQ_K) ? 0 : (td >> 6);
-      for (int kt = 0; kt < k_tiles; ++kt) {
-        const int s = kt % STAGES;
-        const uint32_t ph = (kt / STAGES) & 1;
+      // scale of the block this thread expands at stage kt (0 outside W)
+      auto scale_at = [&](int kt) -> float {
         const int kg = kt0 + kt;
         const int64_t wrow = (BMODE == B_DQ_K) ? static_cast<int64_t>(n0) + row
                                                : static_cast<int64_t>(kg) * 64 + row;
         const int64_t kb = (BMODE == B_DQ_K) ? kg : (n0 / 64 + q);
-        bool valid = wrow < p.w.rows && kb < p.kblocks;
-        if (valid && (wrow * p.kblocks + kb >= p.nblocks)) {
+        if (wrow >= p.w.rows || kb >= p.kblocks) return 0.0f;
+        if (wrow * p.kblocks + kb >= p.nblocks) {
           report(p.st, QLORA_ERR_SHAPE, 201u);
-          valid = false;
+          return 0.0f;
         }
-        // rows or blocks outside W get a zero table, hence zero weights
-        const float sc = valid ? block_scale(p.w, wrow * p.kblocks + kb, mu) : 0.0f;
-        if (!ptx::mbar_wait(&full_tma[s], ph, kTimeoutCycles, abort_flag)) break;
-        uint8_t* sa = smem + s * p.stage_bytes;
-        uint8_t* sb = sa + kA;
-        const uint8_t* codes = sb + p.b_bytes;
+        return block_scale(p.w, wrow * p.kblocks + kb, mu);
+      };
+      float sc_next = k_tiles > 0 ? scale_at(0) : 0.0f;
+      for (int kt = 0; kt < k_tiles; ++kt) {
+        const int s = kt % STAGES;
+        const uint32_t ph = (kt / STAGES) & 1;
+        const int cs = kt % kCodeStages;
+        const float sc = sc_next;
+        if (kt + 1 < k_tiles) sc_next = scale_at(kt + 1);  // prefetch: its loads overlap this stage
+        if (!ptx::mbar_wait(&codes_full[cs], (kt / kCodeStages) & 1, kTimeoutCycles, abort_flag))
+          break;
+        const uint8_t* codes = codes_ring + cs * kCodeBytes;
         const uint8_t* src = (BMODE == B_DQ_K) ? codes + row * 32 : codes + q * 2048 + row * 32;
         const uint4 c0 = *reinterpret_cast<const uint4*>(src);
         const uint4 c1 = *reinterpret_cast<const uint4*>(src + 16);
+        // The next TMA into this slot writes through the async proxy: order
+        // these generic-proxy reads before it, then release the slot.  (Without
+        // the proxy fence the barrier alone let the TMA overwrite codes that
+        // single threads had not yet read: rows of B came out of later tiles.)
+        ptx::fence_proxy_async_smem();
+        ptx::mbar_arrive(&codes_empty[cs]);
         uint32_t L[4], H[4];
         block_tables(lv, sc, L, H);
         const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        // B slot s is free once the MMAs of its previous use have completed
+        if (!ptx::mbar_wait(&empty[s], ph ^ 1, kTimeoutCycles, abort_flag)) break;
+        uint8_t* sb = smem + s * p.stage_bytes + kA;
         uint8_t* dst_row = (BMODE == B_DQ_K) ? sb + row * 128 : sb + q * 8192 + row * 128;
 #pragma unroll
         for (int j = 0; j < 8; ++j)
@@ -453,7 +495,8 @@ template <int BMODE, int STAGES, int MT>
 qlora_status launch_tc(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2,
                        const CUtensorMap& b2, TcArgs p, const LevelTable& t, dim3 grid,
                        cudaStream_t s) {
-  const size_t smem = 1024 + static_cast<size_t>(STAGES) * p.stage_bytes + 256;
+  const size_t smem = 1024 + static_cast<size_t>(STAGES) * p.stage_bytes +
+                      (BMODE != B_TMA_K ? kCodeStages * kCodeBytes : 0) + 256;
   static bool configured = false;
   if (!configured) {
     if (cudaFuncSetAttribute(tc_gemm_kernel<BMODE, STAGES, MT>,
@@ -507,7 +550,7 @@ qlora_status tc_fused_forward(const QView& w, const LevelTable& t, const void* X
   p.k2_tiles = 2 * p.k2_half;
   p.k2_last_steps = ((r - 64 * (p.k2_half - 1)) + 15) / 16;
   p.b_bytes = 32768;
-  p.stage_bytes = 2 * kABytes + 32768 + kCodeBytes;
+  p.stage_bytes = 2 * kABytes + 32768;
   p.tmem_cols = 512;
   p.w = w;
   p.kblocks = static_cast<int>(K / 64);
@@ -537,7 +580,7 @@ qlora_status tc_fused_dgrad(const QView& w, const LevelTable& t, const void* dY,
   p.k2_last_steps = ((r - 64 * (p.k2_half - 1)) + 15) / 16;
   p.b2_mn = 1;
   p.b_bytes = 32768;
-  p.stage_bytes = 2 * kABytes + 32768 + kCodeBytes;
+  p.stage_bytes = 2 * kABytes + 32768;
   p.tmem_cols = 512;
   p.w = w;
   p.kblocks = static_cast<int>(K / 64);
