@@ -34,10 +34,26 @@
 namespace qlora {
 namespace {
 
-constexpr int kThreads = 384;
+// warps 0-3: TMA producer, MMA issuer (and TMEM owner), two idle;
+// warps 4-19: dequantisation in two groups of 256 threads that take alternate
+// stages (more warps in flight to hide the dependent byte-permute chains),
+// then the epilogue
+constexpr int kThreads = 640;
+constexpr int kDqThreads = 256;  // per group
 constexpr int kABytes = 16384;   // 128 rows x 64 bf16
-constexpr int kCodeBytes = 8192;  // codes of one stage: 256 W rows x 32 B (fwd) or 4 x 64 x 32 B (bwd)
-constexpr int kCodeStages = 4;    // depth of the codes ring
+constexpr int kCodeBytes = 8192;  // codes of one k-tile: 256 W rows x 32 B (fwd) or 64 x 128 B (bwd)
+
+// The codes ring: kCG k-tiles per slot, kCSlots slots.  A slot of the
+// decode-sized forward holds 64 contiguous bytes of each of 256 W rows
+// (2 k-tiles), so that every row is read from DRAM in 64-byte pieces.
+template <int BMODE, int MT>
+struct CodesRing {
+  static constexpr bool kWide = (BMODE == B_DQ_K && MT == 1);
+  static constexpr int kCG = kWide ? 2 : 1;
+  static constexpr int kSlots = kWide ? 2 : 4;
+  static constexpr int kSlotBytes = kCG * kCodeBytes;
+  static constexpr int kBytes = (BMODE == B_TMA_K) ? 0 : kSlots * kSlotBytes;
+};
 constexpr long long kTimeoutCycles = 4000000000ll;  // ~2 s at 1.9 GHz
 
 struct TcArgs {
@@ -49,6 +65,7 @@ struct TcArgs {
   int32_t k2_last_steps;  // K=16 steps in the last stage of each half
   int32_t a_mn, b2_mn;
   int32_t b_bytes, stage_bytes, tmem_cols;
+  int32_t a_bytes;        // bytes of A actually loaded per stage (rows beyond M are not fetched)
   QView w;
   int32_t kblocks;        // W.cols / 64
   float alpha;
@@ -149,14 +166,16 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  // [STAGES x (A | B)] [kCodeStages x codes] [barriers]
+  using Ring = CodesRing<BMODE, MT>;
+  constexpr int kCG = Ring::kCG, kCSlots = Ring::kSlots;
+  // [STAGES x (A | B)] [kCSlots x codes] [barriers]
   uint8_t* codes_ring = smem + STAGES * p.stage_bytes;
-  uint64_t* full_a = reinterpret_cast<uint64_t*>(codes_ring + (kDq ? kCodeStages * kCodeBytes : 0));
+  uint64_t* full_a = reinterpret_cast<uint64_t*>(codes_ring + Ring::kBytes);
   uint64_t* full_b = full_a + STAGES;
   uint64_t* empty = full_b + STAGES;
   uint64_t* codes_full = empty + STAGES;
-  uint64_t* codes_empty = codes_full + kCodeStages;
-  uint64_t* accum = codes_empty + kCodeStages;
+  uint64_t* codes_empty = codes_full + kCSlots;
+  uint64_t* accum = codes_empty + kCSlots;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -165,24 +184,27 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   const int n0 = blockIdx.x * p.bn;
   const int kt0 = blockIdx.z * p.k_tiles;
   const int k_tiles = min(p.k_tiles, p.kt_total - kt0);
-  const int total = k_tiles + p.k2_tiles;
+  // with split-K the LoRA extension stages belong to split 0 only
+  const int k2_tiles = blockIdx.z == 0 ? p.k2_tiles : 0;
+  const int total = k_tiles + k2_tiles;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       ptx::mbar_init(&full_a[s], 1);
-      ptx::mbar_init(&full_b[s], 256);
+      ptx::mbar_init(&full_b[s], kDqThreads);
       ptx::mbar_init(&empty[s], 1);
     }
-    for (int s = 0; s < kCodeStages; ++s) {
+    for (int s = 0; s < kCSlots; ++s) {
       ptx::mbar_init(&codes_full[s], 1);
-      ptx::mbar_init(&codes_empty[s], 256);
+      // a slot holding several k-tiles is read by both dequant groups
+      ptx::mbar_init(&codes_empty[s], kCG > 1 ? 2 * kDqThreads : kDqThreads);
     }
     ptx::mbar_init(accum, 1);
     *abort_flag = 0;
     ptx::fence_mbar_init();
     ptx::prefetch_tmap(&tmA);
     ptx::prefetch_tmap(&tmB);
-    if (p.k2_tiles) {
+    if (k2_tiles) {
       ptx::prefetch_tmap(&tmA2);
       ptx::prefetch_tmap(&tmB2);
     }
@@ -199,33 +221,30 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------ TMA producer
     // A (and B when it is bf16) go into stage kt % STAGES once the MMAs of
-    // its previous use are done; the 4-bit codes run up to kCodeStages tiles
-    // ahead in their own ring, freed as soon as the dequant warps read them.
+    // its previous use are done; the 4-bit codes run ahead in their own ring
+    // (groups of kCG k-tiles), freed as soon as the dequant warps read them.
     int issued = 0, kc = 0;
+    const int n_groups = (k_tiles + kCG - 1) / kCG;
     bool ok = true;
     auto issue_codes = [&](int upto) {
-      while (ok && kc < k_tiles && kc < upto) {
-        const int cs = kc % kCodeStages;
-        if (!ptx::mbar_wait(&codes_empty[cs], ((kc / kCodeStages) & 1) ^ 1, kTimeoutCycles,
+      while (ok && kc < n_groups && kc < upto) {
+        const int cs = kc % kCSlots;
+        if (!ptx::mbar_wait(&codes_empty[cs], ((kc / kCSlots) & 1) ^ 1, kTimeoutCycles,
                             abort_flag)) {
           ok = false;
           break;
         }
-        uint8_t* dst = codes_ring + cs * kCodeBytes;
-        const int kg = kt0 + kc;
-        ptx::mbar_arrive_expect_tx(&codes_full[cs], kCodeBytes);
-        if (BMODE == B_DQ_K) {
+        uint8_t* dst = codes_ring + cs * Ring::kSlotBytes;
+        const int kg = kt0 + kc * kCG;
+        ptx::mbar_arrive_expect_tx(&codes_full[cs], Ring::kSlotBytes);
+        if (BMODE == B_DQ_K)
           ptx::tma_load_2d(&tmB, &codes_full[cs], dst, kg * 32, n0);
-        } else {
-          // four 32-byte column slices (one 64-weight block each) of 64 W rows
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            ptx::tma_load_2d(&tmB, &codes_full[cs], dst + q * 2048, n0 / 2 + 32 * q, kg * 64);
-        }
+        else
+          ptx::tma_load_2d(&tmB, &codes_full[cs], dst, n0 / 2, kg * 64);
         ++kc;
       }
     };
-    if (kDq) issue_codes(kCodeStages);
+    if (kDq) issue_codes(kCSlots);
     for (int kt = 0; kt < total && ok; ++kt) {
       const int s = kt % STAGES;
       const uint32_t ph = (kt / STAGES) & 1;
@@ -234,7 +253,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       uint8_t* sb = sa + kA;
       if (kt < k_tiles) {
         const int kg = kt0 + kt;
-        ptx::mbar_arrive_expect_tx(&full_a[s], kA + (kDq ? 0 : p.bn * 128));
+        ptx::mbar_arrive_expect_tx(&full_a[s], p.a_bytes + (kDq ? 0 : p.bn * 128));
         if (p.a_mn) {
           // MN-major A (only with MT == 1): two 64-row halves
           ptx::tma_load_2d(&tmA, &full_a[s], sa, m0, kg * 64);
@@ -249,7 +268,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         const int tt = kt - k_tiles;
         const int k2a = tt * 64;
         const int k2b = (tt % p.k2_half) * 64;
-        ptx::mbar_arrive_expect_tx(&full_a[s], kA + 32768);
+        ptx::mbar_arrive_expect_tx(&full_a[s], p.a_bytes + 32768);
         ptx::tma_load_2d(&tmA2, &full_a[s], sa, k2a, m0);
         if (p.b2_mn) {
 #pragma unroll
@@ -260,13 +279,13 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         }
       }
       ++issued;
-      if (kDq) issue_codes(kt + 1 + kCodeStages);
+      if (kDq) issue_codes(kt / kCG + kCSlots);
     }
     // never leave with copies in flight into this CTA's shared memory
     for (int kt = max(0, issued - STAGES); kt < issued; ++kt)
       ptx::mbar_wait(&full_a[kt % STAGES], (kt / STAGES) & 1, kTimeoutCycles, nullptr);
-    for (int c = max(0, kc - kCodeStages); c < kc; ++c)
-      ptx::mbar_wait(&codes_full[c % kCodeStages], (c / kCodeStages) & 1, kTimeoutCycles, nullptr);
+    for (int c = max(0, kc - kCSlots); c < kc; ++c)
+      ptx::mbar_wait(&codes_full[c % kCSlots], (c / kCSlots) & 1, kTimeoutCycles, nullptr);
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------ MMA issuer
     const uint32_t idesc = ptx::idesc_bf16(128, p.bn, p.a_mn, BMODE == B_DQ_MN ? 1 : 0);
@@ -298,7 +317,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     ptx::umma_commit(accum);
     ptx::mbar_wait(accum, 0, kTimeoutCycles, nullptr);  // MMAs done before TMEM is freed
   } else if (warp >= 4) {
-    const int td = threadIdx.x - 128;
+    const int grp = (threadIdx.x - 128) / kDqThreads;  // dequant group: stages kt % 2 == grp
+    const int td = (threadIdx.x - 128) % kDqThreads;
     if (kDq) {
       // ---------------------------------------------------- dequantisation
       // forward: thread td expands W row n0 + td (one 64-weight block per stage);
@@ -309,38 +329,74 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const float mu = (p.w.dq_shift >= 0) ? __ldg(p.w.mean) : 0.0f;
       const int row = (BMODE == B_DQ_K) ? td : (td & 63);
       const int q = (BMODE == B_DQ_K) ? 0 : (td >> 6);
-      // scale of the block this thread expands at stage kt (0 outside W)
-      auto scale_at = [&](int kt) -> float {
+      // Raw inputs of the scale of the block this thread expands at stage kt:
+      // the int8 code and the group factor (or the fp32 absmax without double
+      // quantisation); `in` is false outside W.  They are loaded four of this
+      // group's stages ahead and combined only when used, so the loads stay in
+      // flight meanwhile (at small M every scale is a first touch from DRAM).
+      struct RawScale {
+        float q, f;
+        bool in;
+      };
+      auto load_scale = [&](int kt) -> RawScale {
+        if (kt >= k_tiles) return RawScale{0.0f, 0.0f, false};
         const int kg = kt0 + kt;
         const int64_t wrow = (BMODE == B_DQ_K) ? static_cast<int64_t>(n0) + row
                                                : static_cast<int64_t>(kg) * 64 + row;
         const int64_t kb = (BMODE == B_DQ_K) ? kg : (n0 / 64 + q);
-        if (wrow >= p.w.rows || kb >= p.kblocks) return 0.0f;
-        if (wrow * p.kblocks + kb >= p.nblocks) {
+        if (wrow >= p.w.rows || kb >= p.kblocks) return RawScale{0.0f, 0.0f, false};
+        const int64_t b = wrow * p.kblocks + kb;
+        if (b >= p.nblocks) {
           report(p.st, QLORA_ERR_SHAPE, 201u);
-          return 0.0f;
+          return RawScale{0.0f, 0.0f, false};
         }
-        return block_scale(p.w, wrow * p.kblocks + kb, mu);
+        if (p.w.dq_shift < 0) return RawScale{1.0f, __ldg(p.w.factors + b), true};
+        return RawScale{static_cast<float>(__ldg(p.w.scale_codes + b)),
+                        __ldg(p.w.factors + (b >> p.w.dq_shift)), true};
       };
-      float sc_next = k_tiles > 0 ? scale_at(0) : 0.0f;
-      for (int kt = 0; kt < k_tiles; ++kt) {
+      const float mu_eff = (p.w.dq_shift >= 0) ? mu : 0.0f;
+      RawScale r0 = load_scale(grp), r1 = load_scale(grp + 2), r2 = load_scale(grp + 4),
+               r3 = load_scale(grp + 6);
+      for (int kt = grp; kt < k_tiles; kt += 2) {
         const int s = kt % STAGES;
         const uint32_t ph = (kt / STAGES) & 1;
-        const int cs = kt % kCodeStages;
-        const float sc = sc_next;
-        if (kt + 1 < k_tiles) sc_next = scale_at(kt + 1);  // prefetch: its loads overlap this stage
-        if (!ptx::mbar_wait(&codes_full[cs], (kt / kCodeStages) & 1, kTimeoutCycles, abort_flag))
+        const int g = kt / kCG, sub = kt % kCG;
+        const int cs = g % kCSlots;
+        // s_hat = fp32(fp32(q * f) + mean) (absmax without double quantisation);
+        // 0 outside W, which makes the whole table 0
+        const float sc = !r0.in ? 0.0f
+                         : (p.w.dq_shift < 0 ? r0.f : __fadd_rn(__fmul_rn(r0.q, r0.f), mu_eff));
+        r0 = r1;
+        r1 = r2;
+        r2 = r3;
+        r3 = load_scale(kt + 8);
+        if (!ptx::mbar_wait(&codes_full[cs], (g / kCSlots) & 1, kTimeoutCycles, abort_flag))
           break;
-        const uint8_t* codes = codes_ring + cs * kCodeBytes;
-        const uint8_t* src = (BMODE == B_DQ_K) ? codes + row * 32 : codes + q * 2048 + row * 32;
-        const uint4 c0 = *reinterpret_cast<const uint4*>(src);
-        const uint4 c1 = *reinterpret_cast<const uint4*>(src + 16);
-        // The next TMA into this slot writes through the async proxy: order
-        // these generic-proxy reads before it, then release the slot.  (Without
-        // the proxy fence the barrier alone let the TMA overwrite codes that
-        // single threads had not yet read: rows of B came out of later tiles.)
-        ptx::fence_proxy_async_smem();
-        ptx::mbar_arrive(&codes_empty[cs]);
+        // this thread's 32 code bytes: fwd decode slots are 64-byte rows, the
+        // backward slot 128-byte rows with the 128B swizzle (16-byte chunk c of
+        // row r at c ^ (r & 7)), the large-M forward slot 32-byte rows
+        const uint8_t* slot = codes_ring + cs * Ring::kSlotBytes;
+        uint4 c0, c1;
+        if (BMODE == B_DQ_K && !Ring::kWide) {
+          c0 = *reinterpret_cast<const uint4*>(slot + row * 32);
+          c1 = *reinterpret_cast<const uint4*>(slot + row * 32 + 16);
+        } else if (BMODE == B_DQ_K) {
+          c0 = *reinterpret_cast<const uint4*>(slot + row * 64 + 32 * sub);
+          c1 = *reinterpret_cast<const uint4*>(slot + row * 64 + 32 * sub + 16);
+        } else {
+          const int chunk = (BMODE == B_DQ_K) ? 2 * sub : 2 * q;
+          c0 = *reinterpret_cast<const uint4*>(slot + row * 128 + 16 * (chunk ^ (row & 7)));
+          c1 = *reinterpret_cast<const uint4*>(slot + row * 128 + 16 * ((chunk + 1) ^ (row & 7)));
+        }
+        // this group's last read of the slot (it reads every other k-tile of it)
+        if (sub + 2 >= kCG || kt + 2 >= k_tiles) {
+          // The next TMA into this slot writes through the async proxy: order
+          // these generic-proxy reads before it, then release the slot.
+          // (Without the proxy fence the barrier alone let the TMA overwrite
+          // codes that single threads had not yet read.)
+          ptx::fence_proxy_async_smem();
+          ptx::mbar_arrive(&codes_empty[cs]);
+        }
         uint32_t L[4], H[4];
         block_tables(lv, sc, L, H);
         const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
@@ -361,14 +417,16 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     if (ok) {
       ptx::tc_fence_after();
       const int quarter = warp & 3;
-      const int group = (warp - 4) >> 2;
+      const int cg = (warp - 4) >> 2;  // 0..3: four warps per TMEM lane quarter
       const int nchunks = p.bn / 16;
-      // MT == 2: group g drains accumulator g; MT == 1: the groups split the columns
-      const int t = (MT == 2) ? group : 0;
-      const int c_first = (MT == 2) ? 0 : group;
-      const int c_step = (MT == 2) ? 1 : 2;
+      // MT == 2: warps cg drain accumulator cg & 1, column half cg >> 1;
+      // MT == 1: the four column groups interleave over 16-column chunks
+      const int t = (MT == 2) ? (cg & 1) : 0;
+      const int c_first = (MT == 2) ? (cg >> 1) * ((nchunks + 1) / 2) : cg;
+      const int c_end = (MT == 2) ? min(nchunks, c_first + (nchunks + 1) / 2) : nchunks;
+      const int c_step = (MT == 2) ? 1 : 4;
       const int64_t row = static_cast<int64_t>(m0) + 128 * t + 32 * quarter + lane;
-      for (int c = c_first; c < nchunks; c += c_step) {
+      for (int c = c_first; c < c_end; c += c_step) {
         uint32_t r[16];
         ptx::tmem_ld_x16(tmem + (static_cast<uint32_t>(32 * quarter) << 16) + t * p.bn + c * 16, r);
         ptx::tmem_ld_wait();
@@ -391,6 +449,28 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 //   o2  bf16  hi = bf16(a2 v) at [i][j] and, if o2_lo > 0, lo = bf16(a2 v - hi) at [i][j + o2_lo]
 //   o3  bf16  the same pair transposed: hi at [j][i], lo at [j + o3_lo][i]
 // hi + lo carries a2 v to about 16 significant bits through bf16 tensor-core operands.
+__device__ __forceinline__ void reduce_store(float v, int64_t i, int j, float* o1, int64_t ld1,
+                                             int trans1, float a1, int acc1, __nv_bfloat16* o2,
+                                             int64_t ld2, float a2, int o2_lo, __nv_bfloat16* o3,
+                                             int64_t ld3, float a3, int o3_lo) {
+  if (o1) {
+    float* dst = trans1 ? o1 + j * ld1 + i : o1 + i * ld1 + j;
+    *dst = acc1 ? *dst + a1 * v : a1 * v;
+  }
+  if (o2) {
+    const float x = a2 * v;
+    const __nv_bfloat16 h = __float2bfloat16_rn(x);
+    o2[i * ld2 + j] = h;
+    if (o2_lo) o2[i * ld2 + j + o2_lo] = __float2bfloat16_rn(x - __bfloat162float(h));
+  }
+  if (o3) {
+    const float x = a3 * v;
+    const __nv_bfloat16 h = __float2bfloat16_rn(x);
+    o3[j * ld3 + i] = h;
+    if (o3_lo) o3[(j + o3_lo) * ld3 + i] = __float2bfloat16_rn(x - __bfloat162float(h));
+  }
+}
+
 __global__ void splitk_reduce_kernel(const float* __restrict__ part, int splits, int64_t rows,
                                      int cols, int pcols, int lo, float* o1, int64_t ld1,
                                      int trans1, float a1, int acc1, __nv_bfloat16* o2, int64_t ld2,
@@ -408,22 +488,35 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ part, int splits,
       v += src[z * split_stride];
       if (lo) v += src[z * split_stride + lo];
     }
-    if (o1) {
-      float* dst = trans1 ? o1 + j * ld1 + i : o1 + i * ld1 + j;
-      *dst = acc1 ? *dst + a1 * v : a1 * v;
+    reduce_store(v, i, j, o1, ld1, trans1, a1, acc1, o2, ld2, a2, o2_lo, o3, ld3, a3, o3_lo);
+  }
+}
+
+// Same reduction with one warp per output: lane l sums splits l, l + 32, ...,
+// then the lanes are combined by a butterfly (a fixed order: deterministic).
+// Used when there are few outputs and many splits.
+__global__ void splitk_reduce_warp_kernel(const float* __restrict__ part, int splits, int64_t rows,
+                                          int cols, int pcols, int lo, float* o1, int64_t ld1,
+                                          int trans1, float a1, int acc1, __nv_bfloat16* o2,
+                                          int64_t ld2, float a2, int o2_lo, __nv_bfloat16* o3,
+                                          int64_t ld3, float a3, int o3_lo) {
+  const int64_t total = rows * cols;
+  const int64_t split_stride = rows * pcols;
+  const int lane = threadIdx.x & 31;
+  for (int64_t e = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; e < total;
+       e += (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5) {
+    const int64_t i = e / cols;
+    const int j = static_cast<int>(e - i * cols);
+    const float* src = part + i * pcols + j;
+    float v = 0.0f;
+    for (int z = lane; z < splits; z += 32) {
+      v += src[z * split_stride];
+      if (lo) v += src[z * split_stride + lo];
     }
-    if (o2) {
-      const float x = a2 * v;
-      const __nv_bfloat16 h = __float2bfloat16_rn(x);
-      o2[i * ld2 + j] = h;
-      if (o2_lo) o2[i * ld2 + j + o2_lo] = __float2bfloat16_rn(x - __bfloat162float(h));
-    }
-    if (o3) {
-      const float x = a3 * v;
-      const __nv_bfloat16 h = __float2bfloat16_rn(x);
-      o3[j * ld3 + i] = h;
-      if (o3_lo) o3[(j + o3_lo) * ld3 + i] = __float2bfloat16_rn(x - __bfloat162float(h));
-    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    if (lane == 0)
+      reduce_store(v, i, j, o1, ld1, trans1, a1, acc1, o2, ld2, a2, o2_lo, o3, ld3, a3, o3_lo);
   }
 }
 
@@ -496,7 +589,7 @@ qlora_status launch_tc(const CUtensorMap& a, const CUtensorMap& b, const CUtenso
                        const CUtensorMap& b2, TcArgs p, const LevelTable& t, dim3 grid,
                        cudaStream_t s) {
   const size_t smem = 1024 + static_cast<size_t>(STAGES) * p.stage_bytes +
-                      (BMODE != B_TMA_K ? kCodeStages * kCodeBytes : 0) + 256;
+                      CodesRing<BMODE, MT>::kBytes + 256;
   static bool configured = false;
   if (!configured) {
     if (cudaFuncSetAttribute(tc_gemm_kernel<BMODE, STAGES, MT>,
@@ -525,6 +618,15 @@ TcArgs base_args(int m, int n, int bn, DeviceStatus* st) {
 
 }  // namespace
 
+// Rows of the activation tile actually fetched: the MMA always runs 128 rows
+// per accumulator, but rows at or beyond M only feed accumulator rows that are
+// never stored, so they need not be loaded.
+uint32_t a_rows(int64_t M, int mt) {
+  const int64_t full = 128 * mt;
+  const int64_t r16 = (M + 15) / 16 * 16;
+  return static_cast<uint32_t>(r16 < full ? r16 : full);
+}
+
 int tc_split_count(int64_t m_tiles, int64_t k_tiles) {
   int64_t s = (2 * 148 + m_tiles - 1) / m_tiles;
   const int64_t max_s = k_tiles / 4 > 0 ? k_tiles / 4 : 1;
@@ -534,63 +636,98 @@ int tc_split_count(int64_t m_tiles, int64_t k_tiles) {
   return static_cast<int>((k_tiles + per - 1) / per);
 }
 
+// Tile shape of the fused kernels: MT 128-row accumulators per CTA and a
+// split of the contraction when the output alone gives too few CTAs.
+FusedShape fused_shape(int64_t M, int64_t n_out, int64_t kt_total) {
+  FusedShape f;
+  const int64_t n_tiles = ceil_div(n_out, 256);
+  f.mt = (M > 128) ? 2 : 1;
+  const int64_t m_tiles = ceil_div(M, 128 * f.mt);
+  f.splits = 1;
+  if (m_tiles * n_tiles < 148) {
+    // one CTA per SM fits (shared memory): stay within a single wave
+    int64_t s = 148 / (m_tiles * n_tiles);
+    const int64_t max_s = kt_total / 2 > 0 ? kt_total / 2 : 1;
+    if (s > max_s) s = max_s;
+    const int64_t per = ceil_div(kt_total, s);
+    f.splits = static_cast<int>(ceil_div(kt_total, per));
+  }
+  return f;
+}
+
+namespace {
+
+template <int BMODE>
+qlora_status launch_fused(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& ma2,
+                          const CUtensorMap& mb2, TcArgs p, const LevelTable& t, int64_t M,
+                          int64_t n_out, const FusedShape& f, cudaStream_t s) {
+  p.k_tiles = static_cast<int>(ceil_div(p.kt_total, f.splits));
+  p.a_bytes = static_cast<int32_t>(a_rows(M, f.mt)) * 128;
+  p.b_bytes = 32768;
+  p.stage_bytes = f.mt * kABytes + 32768;
+  p.tmem_cols = f.mt == 2 ? 512 : 256;
+  dim3 grid(static_cast<unsigned>(ceil_div(n_out, 256)),
+            static_cast<unsigned>(ceil_div(M, 128 * f.mt)), static_cast<unsigned>(f.splits));
+  if (f.mt == 2) return launch_tc<BMODE, 3, 2>(ma, mb, ma2, mb2, p, t, grid, s);
+  return launch_tc<BMODE, 4, 1>(ma, mb, ma2, mb2, p, t, grid, s);
+}
+
+}  // namespace
+
 qlora_status tc_fused_forward(const QView& w, const LevelTable& t, const void* X, int64_t M,
-                              const void* sU, const void* B, int32_t r, void* Y,
-                              DeviceStatus* st, cudaStream_t s) {
+                              const void* sU, const void* B, int32_t r, void* out,
+                              const FusedShape& f, DeviceStatus* st, cudaStream_t s) {
   const int64_t N = w.rows, K = w.cols;
+  const uint32_t rows = a_rows(M, f.mt);
   CUtensorMap ma, mb, ma2, mb2;
-  if (!make_map(&ma, X, true, K, M, K, 64, 256, true) ||
-      !make_map(&mb, w.codes, false, K / 2, N, K / 2, 32, 256, false) ||
-      !make_map(&ma2, sU, true, 2 * lora_span(r), M, 2 * lora_span(r), 64, 256, true) ||
+  if (!make_map(&ma, X, true, K, M, K, 64, rows, true) ||
+      !(f.mt == 1 ? make_map(&mb, w.codes, false, K / 2, N, K / 2, 64, 256, false)
+                  : make_map(&mb, w.codes, false, K / 2, N, K / 2, 32, 256, false)) ||
+      !make_map(&ma2, sU, true, 2 * lora_span(r), M, 2 * lora_span(r), 64, rows, true) ||
       !make_map(&mb2, B, true, r, N, r, 64, 256, true))
     return QLORA_ERR_CUDA;
   TcArgs p = base_args(static_cast<int>(M), static_cast<int>(N), 256, st);
-  p.k_tiles = p.kt_total = static_cast<int>(K / 64);
+  p.kt_total = static_cast<int>(K / 64);
   p.k2_half = (r + 63) / 64;
   p.k2_tiles = 2 * p.k2_half;
   p.k2_last_steps = ((r - 64 * (p.k2_half - 1)) + 15) / 16;
-  p.b_bytes = 32768;
-  p.stage_bytes = 2 * kABytes + 32768;
-  p.tmem_cols = 512;
   p.w = w;
   p.kblocks = static_cast<int>(K / 64);
-  p.out = Y;
-  p.ldo = N;
-  p.out_bf16 = 1;
-  p.out_elems = M * N;
   p.nblocks = N * K / 64;
-  dim3 grid(static_cast<unsigned>(ceil_div(N, 256)), static_cast<unsigned>(ceil_div(M, 256)), 1);
-  return launch_tc<B_DQ_K, 3, 2>(ma, mb, ma2, mb2, p, t, grid, s);
+  p.out = out;
+  p.ldo = N;
+  p.out_bf16 = f.splits == 1 ? 1 : 0;
+  p.split_stride = M * N;
+  p.out_elems = static_cast<int64_t>(f.splits) * M * N;
+  return launch_fused<B_DQ_K>(ma, mb, ma2, mb2, p, t, M, N, f, s);
 }
 
 qlora_status tc_fused_dgrad(const QView& w, const LevelTable& t, const void* dY, int64_t M,
-                            const void* sV, const void* A, int32_t r, void* dX,
-                            DeviceStatus* st, cudaStream_t s) {
+                            const void* sV, const void* A, int32_t r, void* out,
+                            const FusedShape& f, DeviceStatus* st, cudaStream_t s) {
   const int64_t N = w.rows, K = w.cols;
+  const uint32_t rows = a_rows(M, f.mt);
   CUtensorMap ma, mb, ma2, mb2;
-  if (!make_map(&ma, dY, true, N, M, N, 64, 256, true) ||
-      !make_map(&mb, w.codes, false, K / 2, N, K / 2, 32, 64, false) ||
-      !make_map(&ma2, sV, true, 2 * lora_span(r), M, 2 * lora_span(r), 64, 256, true) ||
+  if (!make_map(&ma, dY, true, N, M, N, 64, rows, true) ||
+      !make_map(&mb, w.codes, false, K / 2, N, K / 2, 128, 64, true) ||
+      !make_map(&ma2, sV, true, 2 * lora_span(r), M, 2 * lora_span(r), 64, rows, true) ||
       !make_map(&mb2, A, true, K, r, K, 64, 64, true))
     return QLORA_ERR_CUDA;
   TcArgs p = base_args(static_cast<int>(M), static_cast<int>(K), 256, st);
-  p.k_tiles = p.kt_total = static_cast<int>(ceil_div(N, 64));
+  p.kt_total = static_cast<int>(ceil_div(N, 64));
   p.k2_half = (r + 63) / 64;
   p.k2_tiles = 2 * p.k2_half;
   p.k2_last_steps = ((r - 64 * (p.k2_half - 1)) + 15) / 16;
   p.b2_mn = 1;
-  p.b_bytes = 32768;
-  p.stage_bytes = 2 * kABytes + 32768;
-  p.tmem_cols = 512;
   p.w = w;
   p.kblocks = static_cast<int>(K / 64);
-  p.out = dX;
-  p.ldo = K;
-  p.out_bf16 = 1;
-  p.out_elems = M * K;
   p.nblocks = N * K / 64;
-  dim3 grid(static_cast<unsigned>(ceil_div(K, 256)), static_cast<unsigned>(ceil_div(M, 256)), 1);
-  return launch_tc<B_DQ_MN, 3, 2>(ma, mb, ma2, mb2, p, t, grid, s);
+  p.out = out;
+  p.ldo = K;
+  p.out_bf16 = f.splits == 1 ? 1 : 0;
+  p.split_stride = M * K;
+  p.out_elems = static_cast<int64_t>(f.splits) * M * K;
+  return launch_fused<B_DQ_MN>(ma, mb, ma2, mb2, p, t, M, K, f, s);
 }
 
 // part[z] (m_rows x n_cols fp32) = A . B^T over split z of the contraction; A is
@@ -611,6 +748,7 @@ qlora_status tc_lora_gemm(const void* A, bool a_mn, int64_t m_rows, int64_t kdim
   p.a_mn = a_mn ? 1 : 0;
   p.b_bytes = (bn * 128 + 1023) / 1024 * 1024;
   p.stage_bytes = kABytes + p.b_bytes;
+  p.a_bytes = kABytes;
   p.out = part;
   p.ldo = n_cols;
   p.out_bf16 = 0;
@@ -624,12 +762,20 @@ qlora_status tc_lora_gemm(const void* A, bool a_mn, int64_t m_rows, int64_t kdim
 
 qlora_status splitk_reduce(const ReduceArgs& a, cudaStream_t s) {
   const int64_t total = a.rows * a.cols;
-  const int grid = static_cast<int>(std::min<int64_t>(ceil_div(total, 256), 148 * 8));
   count_launch();
-  splitk_reduce_kernel<<<grid, 256, 0, s>>>(
-      a.part, a.splits, a.rows, a.cols, a.pcols, a.lo, a.o1, a.ld1, a.trans1 ? 1 : 0, a.a1,
-      a.acc1 ? 1 : 0, static_cast<__nv_bfloat16*>(a.o2), a.ld2, a.a2, a.o2_lo,
-      static_cast<__nv_bfloat16*>(a.o3), a.ld3, a.a3, a.o3_lo);
+  if (a.splits >= 16 && total < 32768) {
+    const int grid = static_cast<int>(std::min<int64_t>(ceil_div(total * 32, 256), 148 * 8));
+    splitk_reduce_warp_kernel<<<grid, 256, 0, s>>>(
+        a.part, a.splits, a.rows, a.cols, a.pcols, a.lo, a.o1, a.ld1, a.trans1 ? 1 : 0, a.a1,
+        a.acc1 ? 1 : 0, static_cast<__nv_bfloat16*>(a.o2), a.ld2, a.a2, a.o2_lo,
+        static_cast<__nv_bfloat16*>(a.o3), a.ld3, a.a3, a.o3_lo);
+  } else {
+    const int grid = static_cast<int>(std::min<int64_t>(ceil_div(total, 256), 148 * 8));
+    splitk_reduce_kernel<<<grid, 256, 0, s>>>(
+        a.part, a.splits, a.rows, a.cols, a.pcols, a.lo, a.o1, a.ld1, a.trans1 ? 1 : 0, a.a1,
+        a.acc1 ? 1 : 0, static_cast<__nv_bfloat16*>(a.o2), a.ld2, a.a2, a.o2_lo,
+        static_cast<__nv_bfloat16*>(a.o3), a.ld3, a.a3, a.o3_lo);
+  }
   return after_launch("splitk_reduce", s);
 }
 

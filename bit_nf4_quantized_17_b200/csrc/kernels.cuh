@@ -40,16 +40,25 @@ inline int32_t lora_rows(int32_t r) { return (r + 15) / 16 * 16; }
 
 int tc_split_count(int64_t m_tiles, int64_t k_tiles);
 
+// Shape of a fused launch: mt 128-row accumulators per CTA (1 or 2) and the
+// number of contraction splits (1 = bf16 output written directly; more =
+// fp32 partials out[z] of M x n_out, summed by splitk_reduce).
+struct FusedShape {
+  int mt;
+  int splits;
+};
+FusedShape fused_shape(int64_t M, int64_t n_out, int64_t kt_total);
+
 // Y = X W^T + sU B^T, W dequantised on load; sU (M x 2*lora_span(r) bf16) holds
 // hi = bf16(s X A^T) in columns [0, r) and lo = bf16(s X A^T - hi) from column
 // lora_span(r), zero elsewhere.
 qlora_status tc_fused_forward(const QView& w, const LevelTable& t, const void* X, int64_t M,
-                              const void* sU, const void* B, int32_t r, void* Y,
-                              DeviceStatus* st, cudaStream_t s);
+                              const void* sU, const void* B, int32_t r, void* out,
+                              const FusedShape& f, DeviceStatus* st, cudaStream_t s);
 // dX = dY W + sV A, W dequantised on load; sV laid out like sU, for s dY B.
 qlora_status tc_fused_dgrad(const QView& w, const LevelTable& t, const void* dY, int64_t M,
-                            const void* sV, const void* A, int32_t r, void* dX,
-                            DeviceStatus* st, cudaStream_t s);
+                            const void* sV, const void* A, int32_t r, void* out,
+                            const FusedShape& f, DeviceStatus* st, cudaStream_t s);
 // part[z] (m_rows x n_cols fp32) = A . B^T over split z of the contraction; B has
 // b_rows rows, read as n_cols (rows past b_rows are zero).
 qlora_status tc_lora_gemm(const void* A, bool a_mn, int64_t m_rows, int64_t kdim, int64_t ld_a,
@@ -78,5 +87,19 @@ struct ReduceArgs {
 qlora_status splitk_reduce(const ReduceArgs& a, cudaStream_t s);
 qlora_status transpose_to_bf16(const void* in, bool in_f32, int64_t rows, int cols, int64_t ld_in,
                                void* out, int64_t ld_out, int lo_rows, cudaStream_t s);
+
+// lora_small.cu: LoRA-side kernels for M <= 16 tokens (CUDA cores).
+constexpr int kSmallM = 16;
+int small_chunks(int64_t len);  // partial count of the two reductions below
+// part[z][m][j] (z over 256-wide chunks of d_in, row stride lora_rows(r)) of X A^T
+qlora_status small_down_partial(const void* X, const void* A, int M, int64_t K, int r,
+                                float* part, cudaStream_t s);
+// part[z][m][j] (z over 256-row chunks of d_out) of dY B
+qlora_status small_v_partial(const void* dY, const void* B, int M, int64_t N, int r, float* part,
+                             cudaStream_t s);
+qlora_status small_grad_b(const void* dY, const float* U, int M, int64_t N, int r, float sc,
+                          bool accumulate, float* dB, cudaStream_t s);
+qlora_status small_grad_a(const float* V, const void* X, int M, int64_t K, int r, float sc,
+                          bool accumulate, float* dA, cudaStream_t s);
 
 }  // namespace qlora

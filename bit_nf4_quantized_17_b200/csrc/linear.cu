@@ -5,8 +5,9 @@
 // Backward (same pages, 6 and 3(3)): V = dY B, dX = dY W + s V A,
 // dB = s dY^T U, dA = s V^T X; no gradient for W.
 //
-// Tensor-core path (tcgen05, gemm_tc.cu), taken when M > 16, d_out % 8 == 0
-// and r % 8 == 0 (TMA needs 16-byte row strides):
+// Tensor-core path (tcgen05, gemm_tc.cu), taken when d_out % 8 == 0 and
+// r % 8 == 0 (TMA needs 16-byte row strides); decode-sized M splits the fused
+// kernels over the contraction so that every SM streams weights:
 //   forward   U-GEMM (split-K) -> reduce (U fp32, sU bf16) -> fused
 //             dequant GEMM with the LoRA term as extra K stages          3 launches
 //   backward  U^T (transpose of the given U, or U-GEMM + reduce), B^T,
@@ -32,7 +33,7 @@ float lora_scale(float alpha, int32_t r) { return alpha / static_cast<float>(r);
 
 bool use_tc(int64_t M, int64_t N, int64_t K, int32_t r) {
   (void)K;
-  return M > 16 && M < (int64_t(1) << 30) && N % 8 == 0 && r % 8 == 0;
+  return M >= 1 && M < (int64_t(1) << 30) && N % 8 == 0 && r % 8 == 0;
 }
 
 int64_t pad8(int64_t v) { return (v + 7) / 8 * 8; }
@@ -55,7 +56,7 @@ TcSplits tc_splits(int64_t M, int64_t N, int64_t K) {
 //   backward  U^T [hi ; lo] (2*r16 x M8 bf16) | B^T (r x N bf16) | sV [hi | lo] |
 //             V^T [hi ; lo] | split-K partials
 struct TcLayout {
-  size_t su, part_f, ut, bt, sv, vt, part_b, fwd_end, bwd_end;
+  size_t su, part_f, fused_f, ut, bt, sv, vt, part_b, fused_b, fwd_end, bwd_end;
 };
 
 TcLayout tc_layout(int64_t M, int64_t N, int64_t K, int32_t r) {
@@ -64,7 +65,9 @@ TcLayout tc_layout(int64_t M, int64_t N, int64_t K, int32_t r) {
   TcLayout L{};
   L.su = kStatusBytes;
   L.part_f = L.su + align256(2 * M * 2 * span);
-  L.fwd_end = L.part_f + align256(sizeof(float) * sp.u * M * r16);
+  L.fused_f = L.part_f + align256(sizeof(float) * sp.u * M * r16);
+  const FusedShape ff = fused_shape(M, N, K / 64);
+  L.fwd_end = L.fused_f + (ff.splits > 1 ? align256(sizeof(float) * ff.splits * M * N) : 0);
   L.ut = kStatusBytes;
   L.bt = L.ut + align256(2 * 2 * r16 * mp);
   L.sv = L.bt + align256(2 * r * N);
@@ -72,9 +75,38 @@ TcLayout tc_layout(int64_t M, int64_t N, int64_t K, int32_t r) {
   L.part_b = L.vt + align256(2 * 2 * r16 * mp);
   const int64_t part = std::max(std::max(sp.u * M * r16, sp.v * M * r16),
                                 std::max(sp.db * N * 2 * r16, sp.da * K * 2 * r16));
-  L.bwd_end = L.part_b + align256(sizeof(float) * part);
+  L.fused_b = L.part_b + align256(sizeof(float) * part);
+  const FusedShape fb = fused_shape(M, K, ceil_div(N, 64));
+  L.bwd_end = L.fused_b + (fb.splits > 1 ? align256(sizeof(float) * fb.splits * M * K) : 0);
   return L;
 }
+
+// Workspace of the decode-sized path (M <= 16, tensor-core conditions):
+//   forward   sU [hi | lo] | U-partials | fused partials
+//   backward  sV [hi | lo] | V (fp32) | U (fp32, when recomputed) | partials | fused partials
+struct SmallLayout {
+  size_t su, part_f, fused_f, fwd_end, sv, v, u, part_b, fused_b, bwd_end;
+};
+
+SmallLayout small_layout(int64_t M, int64_t N, int64_t K, int32_t r) {
+  const int64_t r16 = lora_rows(r), span = lora_span(r);
+  SmallLayout L{};
+  L.su = kStatusBytes;
+  L.part_f = L.su + align256(2 * M * 2 * span);
+  L.fused_f = L.part_f + align256(sizeof(float) * small_chunks(K) * M * r16);
+  const FusedShape ff = fused_shape(M, N, K / 64);
+  L.fwd_end = L.fused_f + (ff.splits > 1 ? align256(sizeof(float) * ff.splits * M * N) : 0);
+  L.sv = kStatusBytes;
+  L.v = L.sv + align256(2 * M * 2 * span);
+  L.u = L.v + align256(sizeof(float) * M * r);
+  L.part_b = L.u + align256(sizeof(float) * M * r);
+  L.fused_b = L.part_b + align256(sizeof(float) * std::max(small_chunks(K), small_chunks(N)) * M * r16);
+  const FusedShape fb = fused_shape(M, K, ceil_div(N, 64));
+  L.bwd_end = L.fused_b + (fb.splits > 1 ? align256(sizeof(float) * fb.splits * M * K) : 0);
+  return L;
+}
+
+bool use_small(int64_t M) { return M <= kSmallM; }
 
 ReduceArgs reduce_args(const float* part, int splits, int64_t rows, int cols, int pcols) {
   ReduceArgs a{};
@@ -90,6 +122,12 @@ ReduceArgs reduce_args(const float* part, int splits, int64_t rows, int cols, in
 
 LinearPlan plan_linear(int64_t M, int64_t N, int64_t K, int32_t r) {
   LinearPlan p;
+  if (use_tc(M, N, K, r) && use_small(M)) {
+    SmallLayout L = small_layout(M, N, K, r);
+    p.fwd_workspace = L.fwd_end;
+    p.bwd_workspace = L.bwd_end;
+    return p;
+  }
   if (use_tc(M, N, K, r)) {
     TcLayout L = tc_layout(M, N, K, r);
     p.fwd_workspace = L.fwd_end;
@@ -116,6 +154,33 @@ qlora_status linear_forward(const qlora_nf4& W, const LevelTable& t, const void*
   char* ws = static_cast<char*>(workspace);
   auto* st = reinterpret_cast<DeviceStatus*>(ws);
   const float sc = lora_scale(alpha, r);
+  if (use_tc(M, N, K, r) && use_small(M)) {
+    const SmallLayout L = small_layout(M, N, K, r);
+    const int32_t r16 = lora_rows(r), span = lora_span(r);
+    char* su = ws + L.su;
+    float* part = reinterpret_cast<float*>(ws + L.part_f);
+    if (cudaMemsetAsync(su, 0, sizeof(__nv_bfloat16) * M * 2 * span, s) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+    QLORA_TRY(small_down_partial(X, A, static_cast<int>(M), K, r, part, s));
+    ReduceArgs ra = reduce_args(part, small_chunks(K), M, r, r16);
+    ra.o1 = U_save;
+    ra.ld1 = r;
+    ra.a1 = 1.0f;
+    ra.o2 = su;
+    ra.ld2 = 2 * span;
+    ra.a2 = sc;
+    ra.o2_lo = span;
+    QLORA_TRY(splitk_reduce(ra, s));
+    const FusedShape f = fused_shape(M, N, K / 64);
+    if (f.splits == 1) return tc_fused_forward(w, t, X, M, su, B, r, Y, f, st, s);
+    float* fpart = reinterpret_cast<float*>(ws + L.fused_f);
+    QLORA_TRY(tc_fused_forward(w, t, X, M, su, B, r, fpart, f, st, s));
+    ReduceArgs ry = reduce_args(fpart, f.splits, M, static_cast<int>(N), static_cast<int>(N));
+    ry.o2 = Y;
+    ry.ld2 = N;
+    ry.a2 = 1.0f;
+    return splitk_reduce(ry, s);
+  }
   if (use_tc(M, N, K, r)) {
     const TcLayout L = tc_layout(M, N, K, r);
     const TcSplits sp = tc_splits(M, N, K);
@@ -136,8 +201,17 @@ qlora_status linear_forward(const qlora_nf4& W, const LevelTable& t, const void*
     ra.a2 = sc;
     ra.o2_lo = span;
     QLORA_TRY(splitk_reduce(ra, s));
-    // Y = X W^T + sU B^T in one kernel
-    return tc_fused_forward(w, t, X, M, su, B, r, Y, st, s);
+    // Y = X W^T + sU B^T in one kernel (split over d_in, then summed, when the
+    // output alone would leave SMs idle)
+    const FusedShape f = fused_shape(M, N, K / 64);
+    if (f.splits == 1) return tc_fused_forward(w, t, X, M, su, B, r, Y, f, st, s);
+    float* fpart = reinterpret_cast<float*>(ws + L.fused_f);
+    QLORA_TRY(tc_fused_forward(w, t, X, M, su, B, r, fpart, f, st, s));
+    ReduceArgs ry = reduce_args(fpart, f.splits, M, static_cast<int>(N), static_cast<int>(N));
+    ry.o2 = Y;
+    ry.ld2 = N;
+    ry.a2 = 1.0f;
+    return splitk_reduce(ry, s);
   }
   char* p = ws + kStatusBytes;
   float* u = U_save ? U_save : reinterpret_cast<float*>(p);
@@ -163,6 +237,55 @@ qlora_status linear_backward(const qlora_nf4& W, const LevelTable& t, const void
   const QView w = view_of(W);
   char* ws = static_cast<char*>(workspace);
   auto* st = reinterpret_cast<DeviceStatus*>(ws);
+  if (use_tc(M, N, K, r) && use_small(M)) {
+    const SmallLayout L = small_layout(M, N, K, r);
+    const int32_t r16 = lora_rows(r), span = lora_span(r);
+    const int m = static_cast<int>(M);
+    char* sv = ws + L.sv;
+    float* v = reinterpret_cast<float*>(ws + L.v);
+    float* part = reinterpret_cast<float*>(ws + L.part_b);
+    if (cudaMemsetAsync(sv, 0, sizeof(__nv_bfloat16) * M * 2 * span, s) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+    // V = dY B -> V (fp32) and sV = s V as [hi | lo]
+    QLORA_TRY(small_v_partial(dY, B, m, N, r, part, s));
+    {
+      ReduceArgs ra = reduce_args(part, small_chunks(N), M, r, r16);
+      ra.o1 = v;
+      ra.ld1 = r;
+      ra.a1 = 1.0f;
+      ra.o2 = sv;
+      ra.ld2 = 2 * span;
+      ra.a2 = sc;
+      ra.o2_lo = span;
+      QLORA_TRY(splitk_reduce(ra, s));
+    }
+    if (!U) {
+      float* u = reinterpret_cast<float*>(ws + L.u);
+      QLORA_TRY(small_down_partial(X, A, m, K, r, part, s));
+      ReduceArgs ra = reduce_args(part, small_chunks(K), M, r, r16);
+      ra.o1 = u;
+      ra.ld1 = r;
+      ra.a1 = 1.0f;
+      QLORA_TRY(splitk_reduce(ra, s));
+      U = u;
+    }
+    if (dX) {
+      const FusedShape f = fused_shape(M, K, ceil_div(N, 64));
+      if (f.splits == 1) {
+        QLORA_TRY(tc_fused_dgrad(w, t, dY, M, sv, A, r, dX, f, st, s));
+      } else {
+        float* fpart = reinterpret_cast<float*>(ws + L.fused_b);
+        QLORA_TRY(tc_fused_dgrad(w, t, dY, M, sv, A, r, fpart, f, st, s));
+        ReduceArgs rx = reduce_args(fpart, f.splits, M, static_cast<int>(K), static_cast<int>(K));
+        rx.o2 = dX;
+        rx.ld2 = K;
+        rx.a2 = 1.0f;
+        QLORA_TRY(splitk_reduce(rx, s));
+      }
+    }
+    QLORA_TRY(small_grad_b(dY, U, m, N, r, sc, accumulate, dB, s));
+    return small_grad_a(v, X, m, K, r, sc, accumulate, dA, s);
+  }
   if (use_tc(M, N, K, r)) {
     const TcLayout L = tc_layout(M, N, K, r);
     const TcSplits sp = tc_splits(M, N, K);
@@ -203,8 +326,21 @@ qlora_status linear_backward(const qlora_nf4& W, const LevelTable& t, const void
       ra.o3_lo = r16;
       QLORA_TRY(splitk_reduce(ra, s));
     }
-    // dX = dY W + sV A in one kernel
-    if (dX) QLORA_TRY(tc_fused_dgrad(w, t, dY, M, sv, A, r, dX, st, s));
+    // dX = dY W + sV A in one kernel (split over d_out when needed)
+    if (dX) {
+      const FusedShape f = fused_shape(M, K, ceil_div(N, 64));
+      if (f.splits == 1) {
+        QLORA_TRY(tc_fused_dgrad(w, t, dY, M, sv, A, r, dX, f, st, s));
+      } else {
+        float* fpart = reinterpret_cast<float*>(ws + L.fused_b);
+        QLORA_TRY(tc_fused_dgrad(w, t, dY, M, sv, A, r, fpart, f, st, s));
+        ReduceArgs rx = reduce_args(fpart, f.splits, M, static_cast<int>(K), static_cast<int>(K));
+        rx.o2 = dX;
+        rx.ld2 = K;
+        rx.a2 = 1.0f;
+        QLORA_TRY(splitk_reduce(rx, s));
+      }
+    }
     // dB = s dY^T U: rows d_out, contraction over tokens, hi and lo columns summed
     QLORA_TRY(tc_lora_gemm(dY, true, N, M, N, ut, mp, 2 * r16, 2 * r16, part, sp.db, st, s));
     {

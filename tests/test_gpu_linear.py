@@ -111,6 +111,21 @@ def test_mlp_shapes(mlp, M):
     _run(inp, shape.alpha, rows=rows, w_hat=w_hat)
 
 
+def test_weight_with_zero_double_quant_factors():
+    # every block has the same absmax: each group's centred scales are all 0,
+    # so its factor is 0 and every block dequantises with the mean
+    lv = torch.tensor(oracle.nf4_levels())
+    idx = torch.randint(0, 16, (192, 512), generator=torch.Generator().manual_seed(3))
+    idx[:, ::64] = 15
+    inp, alpha = _inputs(192, 512, 16, 40, 21, b_std=0.05)
+    inp["W"] = (lv[idx] * 0.03125).to(torch.bfloat16)
+    q, *_ = _run(inp, alpha)
+    assert torch.count_nonzero(q.factors) == 0
+    inp1 = dict(inp)
+    inp1["X"], inp1["dY"] = inp["X"][:1].clone(), inp["dY"][:1].clone()
+    _run(inp1, alpha)
+
+
 def test_zero_b_gives_base_output():
     inp, alpha = _inputs(192, 256, 8, 33, 7)
     inp["B"] = torch.zeros_like(inp["B"])
