@@ -44,6 +44,7 @@ TOKENS = 4096
 METRIC = "QLoRA linear fwd+bwd TFLOP/s and NF4 weight GB/s at 1 B200; % of roofline"
 UNIT = "TFLOP/s"
 N_SETS = 3
+CPU_TOKENS = 256   # tokens of the oracle's bounded sample (CPU baseline and reference arm)
 
 
 def fwd_flops(M, N, K, r):
@@ -143,7 +144,7 @@ class ClockSampler:
 # ----------------------------------------------------------- GPU arm -----
 
 class InputSet:
-    def __init__(self, shape, M, seed, rank, dev, Q, WL):
+    def __init__(self, shape, M, seed, rank, dev, Q, WL, dp):
         self.W = WL.weight(shape, seed, dev)
         self.A = WL.lora_a(shape, seed, dev)
         self.B = WL.lora_b(shape, seed, dev)
@@ -159,8 +160,9 @@ class InputSet:
         self.Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
         self.U = torch.empty((M, r), dtype=torch.float32, device=dev)
         self.dX = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
-        self.dA = torch.empty((r, K), dtype=torch.float32, device=dev)
-        self.dB = torch.empty((N, r), dtype=torch.float32, device=dev)
+        # dA and dB are views of one flat buffer: one all-reduce per step
+        self.grads = dp.GradBucket(r, K, N, dev)
+        self.dA, self.dB = self.grads.dA, self.grads.dB
 
 
 def run_step(s, shape, Q, ev=None, world=1):
@@ -175,8 +177,7 @@ def run_step(s, shape, Q, ev=None, world=1):
     if ev is not None:
         ev[2].record()
     if world > 1:
-        torch.distributed.all_reduce(s.dA)
-        torch.distributed.all_reduce(s.dB)
+        s.grads.allreduce()
 
 
 def barrier(world):
@@ -184,12 +185,46 @@ def barrier(world):
         torch.distributed.barrier()
 
 
-def max_over_ranks(value, world, dev):
-    if world == 1:
-        return value
-    t = torch.tensor([value], dtype=torch.float64, device=dev)
-    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    return float(t.item())
+# dram__bytes_read.sum + dram__bytes_write.sum per launch from one ncu capture
+# of the kernel as it is now (profiles/); None once the kernel has changed.
+TRAFFIC = {}
+
+
+def kernel_rooflines(kt, M, N, K, r, peaks):
+    """Per-kernel achieved rate from the library's per-launch CUDA events.
+
+    Algorithmic work per launch (one linear, M tokens):
+      quantise    HBM bytes 2NK (bf16 W) + NK/2 (codes) + 4 NK/64 (fp32 block absmax)
+      fused fwd   FLOPs 2MNK + 2MNr  (base product + LoRA up-projection)
+      fused dgrad FLOPs 2MNK + 2MKr  (dY W + V A)
+      LoRA GEMMs  FLOPs 2MKr (U) + 2MNr (V) + 2MNr (dB) + 2MKr (dA), four launches
+    """
+    from bit_nf4_quantized_17_b200 import qlora as Q
+    nb = -(-N * K // 64)
+    spec = {
+        "quantize_blocks": (Q.QLORA_KERNEL_QUANTIZE, "hbm", 2 * N * K + N * K // 2 + 4 * nb, 1),
+        "fused_fwd": (Q.QLORA_KERNEL_FUSED_FWD, "tensor", 2 * M * N * K + 2 * M * N * r, 1),
+        "fused_dgrad": (Q.QLORA_KERNEL_FUSED_DGRAD, "tensor", 2 * M * N * K + 2 * M * K * r, 1),
+        "lora_gemms": (Q.QLORA_KERNEL_LORA_GEMM, "tensor", 4 * M * K * r + 4 * M * N * r, 4),
+    }
+    out = {}
+    for name, (kind, bound, work, per_step) in spec.items():
+        total_ms, n = kt[kind]
+        if n == 0:
+            continue
+        avg_s = total_ms * 1e-3 / n
+        per_launch = work / per_step
+        if bound == "hbm":
+            achieved, peak, unit = per_launch / avg_s / 1e9, peaks["hbm"], "GB/s"
+            kind_s = f"{peaks['source']} HBM copy bandwidth"
+        else:
+            achieved, peak, unit = per_launch / avg_s / 1e12, peaks["bf16_sustained"], "TFLOP/s"
+            kind_s = f"{peaks['source']} sustained bf16 (kernel timed inside a long step)"
+        out[name] = {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
+                     "frac": round(achieved / peak, 4), "avg_us": round(avg_s * 1e6, 2),
+                     "launches": n, "total_ms": round(total_ms, 4),
+                     "algorithmic_per_launch": per_launch, "peak_kind": kind_s}
+    return out
 
 
 def time_decode(Q, WL, dev, peaks, steps=30, warmup=5):
@@ -216,6 +251,10 @@ def time_decode(Q, WL, dev, peaks, steps=30, warmup=5):
         dB = torch.empty((N, r), dtype=torch.float32, device=dev)
         evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
         for i in range(warmup + steps):
+            if i == warmup:
+                torch.cuda.synchronize()
+                Q.qlora_timing_begin((Q.QLORA_KERNEL_FUSED_FWD, Q.QLORA_KERNEL_FUSED_DGRAD),
+                                     max_launches=4 * steps)
             q = copies[i % 8]
             e = evs[i - warmup] if i >= warmup else None
             if e:
@@ -227,22 +266,36 @@ def time_decode(Q, WL, dev, peaks, steps=30, warmup=5):
             if e:
                 e[2].record()
         torch.cuda.synchronize()
+        kt = Q.qlora_timing_end()
         t_f = statistics.median(e[0].elapsed_time(e[1]) for e in evs) * 1e-3
         t_b = statistics.median(e[1].elapsed_time(e[2]) for e in evs) * 1e-3
         wb = nf4_bytes(N, K)
+        # the fused kernels alone: NF4 bytes + activations in/out + adapter
+        # (algorithmic HBM bytes of one launch) / average launch time
+        fused = {}
+        for name, kind, extra in (("fused_fwd", Q.QLORA_KERNEL_FUSED_FWD, 2 * M * K + 2 * M * N + 2 * N * r),
+                                  ("fused_dgrad", Q.QLORA_KERNEL_FUSED_DGRAD, 2 * M * N + 2 * M * K + 2 * K * r)):
+            ms, n = kt[kind]
+            if n:
+                avg = ms * 1e-3 / n
+                fused[name] = {"avg_us": round(avg * 1e6, 2),
+                               "gbs": round((wb + extra) / avg / 1e9, 1),
+                               "frac_hbm": round((wb + extra) / avg / 1e9 / peaks["hbm"], 4)}
         out[f"M{M}"] = {
             "fwd_us": round(t_f * 1e6, 2), "bwd_us": round(t_b * 1e6, 2),
             "fwd_nf4_gbs": round(wb / t_f / 1e9, 1), "bwd_nf4_gbs": round(wb / t_b / 1e9, 1),
             "fwd_frac_hbm": round(wb / t_f / 1e9 / peaks["hbm"], 4),
             "bwd_frac_hbm": round(wb / t_b / 1e9 / peaks["hbm"], 4),
+            "kernels": fused,
         }
     out["workload"] = "mlp gate/up 11008x4096, r=64, alpha=16; NF4 bytes per pass " \
                       f"{nf4_bytes(N, K)}; 8 rotating weight copies; median of {steps}"
     return out
 
 
-def cpu_oracle_sample(shape, tokens_sample, repeats, WL):
-    """Oracle quantise of the full W + fwd/bwd on `tokens_sample` tokens."""
+def cpu_oracle_sample(shape, tokens_sample, WL, min_seconds=10.0, max_repeats=20):
+    """Oracle quantise of the full W + fwd/bwd on `tokens_sample` tokens,
+    repeated until about `min_seconds` of CPU work (at least 3 repeats)."""
     import oracle
     from threadpoolctl import threadpool_info
     inp = WL.linear_inputs(shape, tokens_sample, 0)
@@ -250,7 +303,7 @@ def cpu_oracle_sample(shape, tokens_sample, repeats, WL):
     f = lambda t: t.float().numpy()
     A, B, X, dY = f(inp["A"]), f(inp["B"]), f(inp["X"]), f(inp["dY"])
     times = []
-    for _ in range(repeats):
+    while len(times) < 3 or (sum(times) < min_seconds and len(times) < max_repeats):
         t0 = time.perf_counter()
         qt = oracle.quantize(W, 64, 256)
         w_hat = oracle.dequantize(qt).reshape(W.shape)
@@ -262,11 +315,13 @@ def cpu_oracle_sample(shape, tokens_sample, repeats, WL):
     flops = fwd_bwd_flops(tokens_sample, shape.d_out, shape.d_in, shape.r)
     return {"value": flops / t / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"oracle quantise of the full 4096x4096 W + fwd/bwd on {tokens_sample} of "
-                      f"the {TOKENS} tokens, median of {repeats}; FLOPs of those tokens / time",
+                      f"the {TOKENS} tokens, median of {len(times)} ({sum(times):.1f} s of CPU "
+                      f"work); FLOPs of those tokens / time",
             "seconds_per_sample": round(t, 3)}
 
 
 def run_ours(args):
+    from bit_nf4_quantized_17_b200 import dp
     from bit_nf4_quantized_17_b200 import qlora as Q
     from bit_nf4_quantized_17_b200 import workloads as WL
 
@@ -282,7 +337,7 @@ def run_ours(args):
     peaks = measured_peaks()
     shape = WL.WORKLOADS[WORKLOAD].linears[0]
     N, K, r, M = shape.d_out, shape.d_in, shape.r, TOKENS
-    sets = [InputSet(shape, M, 100 * i, rank, dev, Q, WL) for i in range(N_SETS)]
+    sets = [InputSet(shape, M, 100 * i, rank, dev, Q, WL, dp) for i in range(N_SETS)]
     torch.cuda.synchronize()
 
     for i in range(args.warmup):
@@ -293,32 +348,47 @@ def run_ours(args):
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     launches0 = Q.qlora_launch_count()
+    # per-kernel CUDA events, recorded by the library on the launching stream
+    # around the two fused kernels (the dominant ones) inside the timed region
+    fused_kinds = (Q.QLORA_KERNEL_FUSED_FWD, Q.QLORA_KERNEL_FUSED_DGRAD)
     with ClockSampler(local) as clk:
         barrier(world)
         torch.cuda.synchronize()
+        Q.qlora_timing_begin(fused_kinds, max_launches=4 * args.steps)
         start.record()
         for i in range(args.steps):
             run_step(sets[i % N_SETS], shape, Q, ev=evs[i], world=world)
         end.record()
         torch.cuda.synchronize()
+        kt = Q.qlora_timing_end()
         barrier(world)
     launches = Q.qlora_launch_count() - launches0
-    elapsed_ms = max_over_ranks(start.elapsed_time(end), world, dev)
+    # the other kernels in a second pass over the same steps (their events
+    # would otherwise add a gap to every launch of the timed region)
+    Q.qlora_timing_begin((Q.QLORA_KERNEL_QUANTIZE, Q.QLORA_KERNEL_LORA_GEMM),
+                         max_launches=8 * args.steps)
+    for i in range(args.steps):
+        run_step(sets[i % N_SETS], shape, Q, world=world)
+    torch.cuda.synchronize()
+    kt2 = Q.qlora_timing_end()
+    for k in (Q.QLORA_KERNEL_QUANTIZE, Q.QLORA_KERNEL_LORA_GEMM):
+        kt[k] = kt2[k]
+    elapsed_ms = dp.max_over_ranks(start.elapsed_time(end), dev)
     ms_per_step = elapsed_ms / args.steps
     flops_step = fwd_bwd_flops(M, N, K, r)
     value = flops_step * world / (ms_per_step * 1e-3) / 1e12
     t_fwd = statistics.mean(e[0].elapsed_time(e[1]) for e in evs) * 1e-3
     t_bwd = statistics.mean(e[1].elapsed_time(e[2]) for e in evs) * 1e-3
 
-    # roofline of the dominant kernel: the fused forward GEMM, timed as the
-    # whole forward call (its LoRA pre-GEMM included, so "achieved" is a lower bound)
-    achieved = fwd_flops(M, N, K, r) / t_fwd / 1e12
-    roofline = {"bound": "tensor", "achieved": round(achieved, 2),
-                "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
-                "frac": round(achieved / peaks["bf16_sustained"], 4),
-                "traffic": None,
-                "kernel": "forward call (LoRA pre-GEMM + fused dequant GEMM)",
-                "peak_kind": f"{peaks['source']} sustained bf16 (kernel timed inside a long step)"}
+    kernels = kernel_rooflines(kt, M, N, K, r, peaks)
+    # the roofline line is the kernel with the largest share of device time
+    dominant = max(kernels, key=lambda k: kernels[k]["total_ms"])
+    d = kernels[dominant]
+    roofline = {"bound": d["bound"], "achieved": d["achieved"], "peak": d["peak"],
+                "unit": d["unit"], "frac": d["frac"], "traffic": TRAFFIC.get(dominant),
+                "kernel": dominant, "avg_launch_us": d["avg_us"],
+                "algorithmic_per_launch": d["algorithmic_per_launch"],
+                "peak_kind": d["peak_kind"]}
 
     # end to end: host (pinned) inputs copied in, results copied out, every step
     e2e = None
@@ -347,7 +417,7 @@ def run_ours(args):
             e2e_step()
         e1.record()
         torch.cuda.synchronize()
-        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / args.steps
+        e2e_ms = dp.max_over_ranks(e0.elapsed_time(e1), dev) / args.steps
         e2e = {"value": round(flops_step * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
                "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h,
@@ -360,7 +430,7 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
-        cpu = cpu_oracle_sample(shape, 64, 3, WL)
+        cpu = cpu_oracle_sample(shape, CPU_TOKENS, WL)
 
     if world > 1:
         torch.distributed.barrier()
@@ -379,7 +449,7 @@ def run_ours(args):
         "fwd_tflops": round(fwd_flops(M, N, K, r) / t_fwd / 1e12, 2),
         "bwd_tflops": round((fwd_bwd_flops(M, N, K, r) - fwd_flops(M, N, K, r)) / t_bwd / 1e12, 2),
         "frac_of_bf16_peak": round(value / world / peaks["bf16_sustained"], 4),
-        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": launches, "clocks": clk.summary(), "decode": decode,
         "peaks": peaks,
     }
@@ -399,7 +469,7 @@ def run_reference(args):
     from bit_nf4_quantized_17_b200 import workloads as WL
 
     shape = WL.WORKLOADS[WORKLOAD].linears[0]
-    ms = 32
+    ms = CPU_TOKENS
     inp = WL.linear_inputs(shape, ms, 0)
     W = inp["W"].float().numpy()
     f = lambda t: t.float().numpy()

@@ -5,6 +5,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "internal.cuh"
 #include "kernels.cuh"
@@ -14,9 +15,38 @@ using namespace qlora;
 
 namespace {
 std::atomic<uint64_t> g_launches{0};
+
+// State of qlora_timing_begin/end: event pairs, the kind of each, how many used.
+struct Timing {
+  std::mutex mu;
+  std::atomic<bool> on{false};
+  uint32_t mask = 0;
+  std::vector<cudaEvent_t> ev;  // 2 per launch: start, stop
+  std::vector<int> kind;
+  int used = 0;
+  bool open = false;  // a start was recorded, its stop not yet
+};
+Timing g_timing;
 }  // namespace
 
 void qlora::count_launch(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+void qlora::timing_mark(int kind, cudaStream_t s, bool start) {
+  if (!g_timing.on.load(std::memory_order_acquire)) return;
+  std::lock_guard<std::mutex> lock(g_timing.mu);
+  if (!g_timing.on.load() || !(g_timing.mask >> kind & 1u)) return;
+  const int cap = static_cast<int>(g_timing.kind.size());
+  if (start) {
+    if (g_timing.used >= cap) return;
+    if (cudaEventRecord(g_timing.ev[2 * g_timing.used], s) == cudaSuccess) {
+      g_timing.kind[g_timing.used] = kind;
+      g_timing.open = true;
+    }
+  } else if (g_timing.open) {
+    g_timing.open = false;
+    if (cudaEventRecord(g_timing.ev[2 * g_timing.used + 1], s) == cudaSuccess) ++g_timing.used;
+  }
+}
 
 qlora_status qlora::after_launch(const char* kernel, cudaStream_t s) {
   static const bool sync_check = [] {
@@ -224,5 +254,56 @@ qlora_status qlora_check(void* workspace, void* stream) {
 }
 
 uint64_t qlora_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+qlora_status qlora_timing_begin(uint32_t kind_mask, int32_t max_launches) {
+  if (max_launches < 1 || max_launches > 65536) return QLORA_ERR_SHAPE;
+  std::lock_guard<std::mutex> lock(g_timing.mu);
+  if (g_timing.on.load()) return QLORA_ERR_UNSUPPORTED;
+  g_timing.ev.assign(2 * static_cast<size_t>(max_launches), nullptr);
+  for (auto& e : g_timing.ev) {
+    if (cudaEventCreate(&e) != cudaSuccess) {
+      for (auto& d : g_timing.ev)
+        if (d) cudaEventDestroy(d);
+      g_timing.ev.clear();
+      return QLORA_ERR_CUDA;
+    }
+  }
+  g_timing.kind.assign(static_cast<size_t>(max_launches), -1);
+  g_timing.mask = kind_mask;
+  g_timing.used = 0;
+  g_timing.open = false;
+  g_timing.on.store(true, std::memory_order_release);
+  return QLORA_OK;
+}
+
+qlora_status qlora_timing_end(float* ms, int32_t* launches) {
+  std::lock_guard<std::mutex> lock(g_timing.mu);
+  if (!g_timing.on.load()) return QLORA_ERR_UNSUPPORTED;
+  g_timing.on.store(false, std::memory_order_release);
+  float total[QLORA_KERNEL_KINDS] = {};
+  int32_t count[QLORA_KERNEL_KINDS] = {};
+  qlora_status st = QLORA_OK;
+  for (int i = 0; i < g_timing.used && st == QLORA_OK; ++i) {
+    float t = 0.0f;
+    if (cudaEventSynchronize(g_timing.ev[2 * i + 1]) != cudaSuccess ||
+        cudaEventElapsedTime(&t, g_timing.ev[2 * i], g_timing.ev[2 * i + 1]) != cudaSuccess) {
+      st = QLORA_ERR_CUDA;
+      break;
+    }
+    const int k = g_timing.kind[i];
+    if (k >= 0 && k < QLORA_KERNEL_KINDS) {
+      total[k] += t;
+      ++count[k];
+    }
+  }
+  for (auto& e : g_timing.ev) cudaEventDestroy(e);
+  g_timing.ev.clear();
+  g_timing.kind.clear();
+  for (int k = 0; k < QLORA_KERNEL_KINDS; ++k) {
+    if (ms) ms[k] = total[k];
+    if (launches) launches[k] = count[k];
+  }
+  return st;
+}
 
 }  // extern "C"

@@ -599,7 +599,12 @@ qlora_status launch_tc(const CUtensorMap& a, const CUtensorMap& b, const CUtenso
     configured = true;
   }
   count_launch();
+  constexpr int kind = BMODE == B_TMA_K   ? QLORA_KERNEL_LORA_GEMM
+                       : BMODE == B_DQ_K ? QLORA_KERNEL_FUSED_FWD
+                                         : QLORA_KERNEL_FUSED_DGRAD;
+  timing_mark(kind, s, true);
   tc_gemm_kernel<BMODE, STAGES, MT><<<grid, kThreads, smem, s>>>(a, b, a2, b2, p, t);
+  timing_mark(kind, s, false);
   return after_launch(BMODE == B_TMA_K ? "tc_gemm(lora)" : BMODE == B_DQ_K ? "tc_gemm(fwd)" : "tc_gemm(dgrad)", s);
 }
 

@@ -40,6 +40,11 @@ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 // abi.cu: every kernel launch site calls this once per launch.
 void count_launch(unsigned n = 1);
 
+// abi.cu: kernel timing hook.  A launch site of a timed kind calls it with
+// start = true just before its launch and start = false just after; both are
+// no-ops unless qlora_timing_begin enabled that kind.
+void timing_mark(int kind, cudaStream_t s, bool start);
+
 // abi.cu: status of the launch just enqueued.  With the environment variable
 // QLORA_SYNC_CHECK=1 the stream is synchronised after every launch and a
 // failing kernel is named on stderr (a debugging aid; off by default).

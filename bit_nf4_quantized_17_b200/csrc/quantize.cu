@@ -244,6 +244,7 @@ void launch_blocks(int bs, const T* w, int64_t n, const LevelTable& t, uint8_t* 
   const int64_t nb = ceil_div(n, bs);
   const int grid = grid_for(nb, 8, 148 * 16);
   count_launch();
+  timing_mark(QLORA_KERNEL_QUANTIZE, s, true);
   switch (bs) {
     case 64: quantize_blocks_kernel<T, 64><<<grid, 256, 0, s>>>(w, n, t, codes, absmax, gmax, st); break;
     case 128: quantize_blocks_kernel<T, 128><<<grid, 256, 0, s>>>(w, n, t, codes, absmax, gmax, st); break;
@@ -251,6 +252,7 @@ void launch_blocks(int bs, const T* w, int64_t n, const LevelTable& t, uint8_t* 
     case 512: quantize_blocks_kernel<T, 512><<<grid, 256, 0, s>>>(w, n, t, codes, absmax, gmax, st); break;
     default: quantize_blocks_kernel<T, 1024><<<grid, 256, 0, s>>>(w, n, t, codes, absmax, gmax, st); break;
   }
+  timing_mark(QLORA_KERNEL_QUANTIZE, s, false);
 }
 
 }  // namespace

@@ -31,6 +31,12 @@ QLORA_BF16 = 1
 QLORA_TABLE_NF4 = 0
 QLORA_TABLE_UNIFORM = 1
 
+QLORA_KERNEL_QUANTIZE = 0
+QLORA_KERNEL_FUSED_FWD = 1
+QLORA_KERNEL_FUSED_DGRAD = 2
+QLORA_KERNEL_LORA_GEMM = 3
+QLORA_KERNEL_KINDS = 4
+
 _DTYPE = {torch.float32: QLORA_F32, torch.bfloat16: QLORA_BF16}
 
 
@@ -77,6 +83,9 @@ def lib():
                                                 i32, vp, sz, vp]),
             "qlora_check": (ctypes.c_int, [vp, vp]),
             "qlora_launch_count": (ctypes.c_uint64, []),
+            "qlora_timing_begin": (ctypes.c_int, [ctypes.c_uint32, i32]),
+            "qlora_timing_end": (ctypes.c_int, [ctypes.POINTER(ctypes.c_float),
+                                                ctypes.POINTER(ctypes.c_int32)]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -236,6 +245,22 @@ def qlora_linear_bwd(q, A, B, alpha, X, U, dY, dX=None, dA=None, dB=None, accumu
 
 def qlora_launch_count():
     return int(lib().qlora_launch_count())
+
+
+def qlora_timing_begin(kinds, max_launches=4096):
+    """Start timing every launch of the given kernel kinds (QLORA_KERNEL_*)."""
+    mask = 0
+    for k in kinds:
+        mask |= 1 << int(k)
+    _ok(lib().qlora_timing_begin(mask, int(max_launches)), "qlora_timing_begin")
+
+
+def qlora_timing_end():
+    """Stop timing; {kind: (total ms, launches)} for every kind."""
+    ms = (ctypes.c_float * QLORA_KERNEL_KINDS)()
+    n = (ctypes.c_int32 * QLORA_KERNEL_KINDS)()
+    _ok(lib().qlora_timing_end(ms, n), "qlora_timing_end")
+    return {k: (float(ms[k]), int(n[k])) for k in range(QLORA_KERNEL_KINDS)}
 
 
 def qlora_check(workspace, stream=None):

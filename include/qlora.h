@@ -175,6 +175,29 @@ qlora_status qlora_check(void* workspace, void* stream);
  * threads, all calls; memsets not counted).  Host only, never fails. */
 uint64_t qlora_launch_count(void);
 
+/* Kernel timing (measurement aid).  Between qlora_timing_begin and
+ * qlora_timing_end the library records a pair of CUDA events on the launching
+ * stream around every launch of the kernel kinds in `kind_mask` (bit k set =
+ * kind k), for at most `max_launches` launches in all (later ones are not
+ * timed).  qlora_timing_end waits for the recorded events, writes the summed
+ * device time in milliseconds and the launch count of each kind to
+ * ms[QLORA_KERNEL_KINDS] and launches[QLORA_KERNEL_KINDS] (either may be
+ * NULL), and releases the events.  The events are library-owned host
+ * objects; no device memory is allocated.  Launches from several host
+ * threads at once are not supported while timing is on.
+ * Errors: QLORA_ERR_SHAPE for max_launches outside [1, 65536],
+ * QLORA_ERR_UNSUPPORTED for begin while timing is already on or end while it
+ * is off, QLORA_ERR_CUDA if an event cannot be created or read. */
+typedef enum {
+  QLORA_KERNEL_QUANTIZE = 0,     /* block absmax, nearest level, nibble packing */
+  QLORA_KERNEL_FUSED_FWD = 1,    /* fused dequant GEMM of the forward pass */
+  QLORA_KERNEL_FUSED_DGRAD = 2,  /* fused dequant GEMM of dX */
+  QLORA_KERNEL_LORA_GEMM = 3,    /* tensor-core rank-r GEMMs (U, V, dA, dB) */
+  QLORA_KERNEL_KINDS = 4
+} qlora_kernel_kind;
+qlora_status qlora_timing_begin(uint32_t kind_mask, int32_t max_launches);
+qlora_status qlora_timing_end(float* ms, int32_t* launches);
+
 #ifdef __cplusplus
 }
 #endif

@@ -137,3 +137,12 @@ def test_status_strings():
     for s in range(9):
         assert Q.qlora_status_string(s)
     assert Q.qlora_status_string(99) == "unknown status"
+
+
+def test_timing_hook_rejects_bad_requests_without_cuda():
+    L = Q.lib()
+    # out-of-range launch budgets are refused before any event is created
+    assert L.qlora_timing_begin(0x3, 0) == Q.QLORA_ERR_SHAPE
+    assert L.qlora_timing_begin(0x3, 65537) == Q.QLORA_ERR_SHAPE
+    # ending while timing is off
+    assert L.qlora_timing_end(None, None) == Q.QLORA_ERR_UNSUPPORTED

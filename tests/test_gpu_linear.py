@@ -111,6 +111,29 @@ def test_mlp_shapes(mlp, M):
     _run(inp, shape.alpha, rows=rows, w_hat=w_hat)
 
 
+def _stack_linear(workload, j, layer, n_rows=32):
+    """Linear j of layer `layer` of a stack workload at its token count, its
+    seeds as the stack draws them; Y and dX checked on sampled token rows."""
+    wl = WL.WORKLOADS[workload]
+    shape, M = wl.linears[j], wl.tokens[0]
+    inp = WL.linear_inputs(shape, M, WL.stack_seed(layer, j))
+    rows = np.sort(np.random.default_rng(7 * layer + j).choice(M, n_rows, replace=False))
+    rows = np.concatenate([[0], rows, [M - 1]])
+    _run(inp, shape.alpha, rows=rows)
+
+
+@pytest.mark.parametrize("j", range(7), ids=[n for n, _, _ in WL.LLAMA7B_LINEARS])
+def test_stack_7b_layer_linears(j):
+    # first and last layer of the 32-layer stack (different seeds)
+    _stack_linear("stack_7b", j, 0)
+    _stack_linear("stack_7b", j, 31, n_rows=8)
+
+
+@pytest.mark.parametrize("j", [0, 4, 6], ids=["q_8192", "gate_22016x8192", "down_8192x22016"])
+def test_stack_65b_linear_shapes(j):
+    _stack_linear("stack_65b", j, 0)
+
+
 def test_weight_with_zero_double_quant_factors():
     # every block has the same absmax: each group's centred scales are all 0,
     # so its factor is 0 and every block dequantises with the mean
