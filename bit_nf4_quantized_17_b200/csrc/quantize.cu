@@ -8,10 +8,11 @@
 //
 // Launch sequence of qlora_quantize (all on the caller's stream):
 //   1. memset of the reduction words in the workspace
-//   2. quantize_blocks_kernel   one warp per block: warp-shuffle absmax,
-//                               IEEE division, 4-step branch-free search of
-//                               the decision thresholds, nibble packing; CTA
-//                               max of the scales -> one atomicMax per CTA
+//   2. quantize_blocks_kernel   16 (or 32) weights per thread, one block per
+//                               4..32 lanes: shuffle absmax, nearest level by
+//                               a cell lookup (IEEE division where the lookup
+//                               cannot decide), nibble packing; CTA max of
+//                               the scales -> one atomicMax per CTA
 //   3. scale_sum_kernel         fixed-point sum of the scales (integer
 //                               atomics: the result is order-independent)
 //   4. dq_groups_kernel         one CTA per group: centred scales, group
@@ -20,6 +21,8 @@
 // `factors`.
 #include <cuda_bf16.h>
 
+#include <cstring>
+
 #include "internal.cuh"
 
 namespace qlora {
@@ -27,83 +30,225 @@ namespace {
 
 constexpr int kMeanFracBits = 32;
 
-__device__ __forceinline__ int nearest_index(float x, const float* thr) {
-  int i = (x > thr[7]) ? 8 : 0;
-  i += (x > thr[i + 3]) ? 4 : 0;
-  i += (x > thr[i + 1]) ? 2 : 0;
-  i += (x > thr[i]) ? 1 : 0;
-  return i;
+// Nearest-level search.  The index of x = RN(w / s) is the number of
+// decision thresholds below it (ties go to the lower level).  The quantiser
+// finds it without dividing for almost every weight:
+//   x' = RN(w * RN(1/s)) lies within 1.5e-7 of x (|x| <= 1 and s a normal
+//   float: two roundings of relative size 2^-24 each, plus the rounding of x);
+//   c = round(32 x') + 32 picks one of 65 cells of width 1/32 covering
+//   [-1, 1] (computed exactly by one FMA into the low mantissa bits of
+//   1.5 * 2^23); every gap between thresholds of the two tables is wider than
+//   a cell (NF4: 0.046, uniform: 0.133), so a cell widened by kCellPad on each
+//   side holds at most one threshold t_c (2.0 when it holds none);
+//   index = (number of thresholds below the widened cell) + (x' > t_c).
+// The comparison of x' with t_c agrees with that of x whenever
+// |x' - t_c| > kNear; otherwise, and for blocks whose scale is 0, subnormal,
+// huge or not finite, the chunk is redone with IEEE division and a comparison
+// against every threshold.
+//
+// Arithmetic form (mostly FMA-pipe work): step = sat((x' - t_c) * 2^126) is
+// 1.0 or 0.0 outside the near band; 2^23 + count + step has the index in its
+// low mantissa bits, and an integer multiply-add places those bits at the
+// weight's nibble (the constant 2^23 bits cancel: see kPackBias).
+constexpr int kCells = 65;
+constexpr double kCellPad = 1e-6;
+constexpr float kNear = 1e-6f;
+// 32-bit words of the float 2^23 (+ index), shifted to nibbles 0 and 1, summed
+// mod 2^32 (higher nibbles shift the constant out): 0x4B000000 + 0xB0000000.
+constexpr uint32_t kPackBias = 0xFB000000u;
+
+struct CellLut {
+  float2 e[kCells];  // x: t_c, y: 2^23 + number of thresholds below the cell
+};
+
+bool make_cell_lut(const LevelTable& tab, CellLut* out) {
+  for (int c = 0; c < kCells; ++c) {
+    const double lo = (c - 32 - 0.5) / 32.0 - kCellPad;
+    const double hi = (c - 32 + 0.5) / 32.0 + kCellPad;
+    int below = 0, inside = -1, n_inside = 0;
+    for (int k = 0; k < 15; ++k) {
+      const double t = tab.thr[k];
+      if (t < lo) {
+        ++below;
+      } else if (t <= hi) {
+        inside = k;
+        ++n_inside;
+      }
+    }
+    if (n_inside > 1) return false;
+    out->e[c].x = n_inside ? tab.thr[inside] : 2.0f;
+    out->e[c].y = 8388608.0f + static_cast<float>(below);
+  }
+  return true;
 }
 
-__device__ __forceinline__ float to_f32(float v) { return v; }
-__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+// Raw words of E consecutive weights at e0 (bf16: two per 32-bit word, the
+// even element in the low half); zeros at and beyond n.
+template <typename T, int E>
+struct Raw {
+  static constexpr int kWords = sizeof(T) == 4 ? E : E / 2;
+  uint32_t u[kWords];
+};
 
-template <typename T>
-__device__ __forceinline__ void load_pair(const T* __restrict__ w, int64_t e, int64_t n,
-                                          float& a, float& b) {
-  if (e + 1 < n) {
-    if constexpr (sizeof(T) == 4) {
-      float2 v = __ldg(reinterpret_cast<const float2*>(w + e));
-      a = v.x;
-      b = v.y;
-    } else {
-      __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(w + e);
-      a = __low2float(v);
-      b = __high2float(v);
+template <typename T, int E>
+__device__ __forceinline__ void load_raw(const T* __restrict__ w, int64_t e0, int64_t n,
+                                         Raw<T, E>& r) {
+  if (e0 + E <= n) {
+#pragma unroll
+    for (int i = 0; i < Raw<T, E>::kWords / 4; ++i) {
+      const uint4 q = __ldg(reinterpret_cast<const uint4*>(w + e0) + i);
+      r.u[4 * i] = q.x;
+      r.u[4 * i + 1] = q.y;
+      r.u[4 * i + 2] = q.z;
+      r.u[4 * i + 3] = q.w;
     }
   } else {
-    a = (e < n) ? to_f32(w[e]) : 0.0f;
-    b = 0.0f;
+    const uint32_t* wb = reinterpret_cast<const uint32_t*>(w);
+#pragma unroll
+    for (int i = 0; i < Raw<T, E>::kWords; ++i) {
+      uint32_t x = 0u;
+      if constexpr (sizeof(T) == 4) {
+        if (e0 + i < n) x = wb[e0 + i];
+      } else {
+        const uint16_t* h = reinterpret_cast<const uint16_t*>(w);
+        if (e0 + 2 * i < n) x = h[e0 + 2 * i];
+        if (e0 + 2 * i + 1 < n) x |= static_cast<uint32_t>(h[e0 + 2 * i + 1]) << 16;
+      }
+      r.u[i] = x;
+    }
   }
 }
 
+template <typename T, int E>
+__device__ __forceinline__ void unpack_raw(const Raw<T, E>& r, float* v) {
+#pragma unroll
+  for (int i = 0; i < Raw<T, E>::kWords; ++i) {
+    if constexpr (sizeof(T) == 4) {
+      v[i] = __uint_as_float(r.u[i]);
+    } else {
+      v[2 * i] = __uint_as_float(r.u[i] << 16);
+      v[2 * i + 1] = __uint_as_float(r.u[i] & 0xffff0000u);
+    }
+  }
+}
+
+// max(a, |b|), NaN if either is NaN
+__device__ __forceinline__ float max_abs_nan(float a, float b) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(fabsf(b)));
+  return r;
+}
+
+// One thread per E consecutive weights (16-byte loads), BS / E threads per
+// block, all within one warp: the block absmax is a shuffle reduction over
+// those threads.  Codes go out as one 8- or 16-byte store per thread; the
+// first thread of each block writes its scale.  The next chunk's words are
+// loaded before the current one is processed.
 template <typename T, int BS>
 __global__ void __launch_bounds__(256)
-quantize_blocks_kernel(const T* __restrict__ w, int64_t n, LevelTable tab,
+quantize_blocks_kernel(const T* __restrict__ w, int64_t n, LevelTable tab, CellLut cells,
                        uint8_t* __restrict__ codes, float* __restrict__ absmax,
                        unsigned int* __restrict__ gmax_bits, DeviceStatus* st) {
-  constexpr int kPairs = BS / 64;  // element pairs per lane per block
-  __shared__ float thr[16];
+  constexpr int E = BS <= 512 ? 16 : 32;  // weights per thread
+  constexpr int TPB = BS / E;             // threads per block: 4 .. 32
+  constexpr int W = E / 8;                // 32-bit words of codes per thread
+  // cell table replicated per lane (entry c of lane l at c * 32 + l): a warp's
+  // 8-byte reads take the minimum two shared-memory wavefronts
+  __shared__ float2 lut[kCells * 32];
   __shared__ unsigned int cta_max;
-  if (threadIdx.x < 16) thr[threadIdx.x] = tab.thr[threadIdx.x];
+  for (int i = threadIdx.x; i < kCells * 32; i += blockDim.x) lut[i] = cells.e[i >> 5];
   if (threadIdx.x == 0) cta_max = 0u;
   __syncthreads();
 
   const int lane = threadIdx.x & 31;
-  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  const int64_t nb = (n + BS - 1) / BS;
-  float seen_max = 0.0f;
+  const float2* my_lut = lut + lane;
+  const int64_t n_chunks = (n + E - 1) / E;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  float seen = 0.0f;  // largest finite scale
   bool nonfinite = false;
 
-  for (int64_t b = warp; b < nb; b += nwarps) {
-    const int64_t base = b * BS;
-    float v[2 * kPairs];
+  // the trip count is the same for every lane of a warp (shuffles inside)
+  int64_t wc = static_cast<int64_t>(blockIdx.x) * blockDim.x + (threadIdx.x & ~31);
+  Raw<T, E> cur;
+  if (wc < n_chunks) load_raw<T, E>(w, (wc + lane) * E, n, cur);
+  for (; wc < n_chunks; wc += stride) {
+    const int64_t e0 = (wc + lane) * E;
+    Raw<T, E> nxt;
+    if (wc + stride < n_chunks) load_raw<T, E>(w, (wc + stride + lane) * E, n, nxt);
+    float v[E];
+    unpack_raw<T, E>(cur, v);
     float a = 0.0f;
 #pragma unroll
-    for (int j = 0; j < kPairs; ++j) {
-      load_pair(w, base + 64 * j + 2 * lane, n, v[2 * j], v[2 * j + 1]);
-      nonfinite |= !isfinite(v[2 * j]) || !isfinite(v[2 * j + 1]);
-      a = fmaxf(a, fmaxf(fabsf(v[2 * j]), fabsf(v[2 * j + 1])));
-    }
+    for (int j = 0; j < E; ++j) a = max_abs_nan(a, v[j]);
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
-#pragma unroll
-    for (int j = 0; j < kPairs; ++j) {
-      const int64_t e = base + 64 * j + 2 * lane;
-      if (e >= n) continue;
-      float x0 = (a > 0.0f) ? __fdiv_rn(v[2 * j], a) : 0.0f;
-      float x1 = (a > 0.0f) ? __fdiv_rn(v[2 * j + 1], a) : 0.0f;
-      int i0 = nearest_index(x0, thr);
-      int i1 = (e + 1 < n) ? nearest_index(x1, thr) : 0;
-      codes[e >> 1] = static_cast<uint8_t>(i0 | (i1 << 4));
+    for (int off = 1; off < TPB; off <<= 1) {
+      const float o = __shfl_xor_sync(0xffffffffu, a, off);
+      asm("max.NaN.f32 %0, %0, %1;" : "+f"(a) : "f"(o));
     }
-    if (lane == 0) absmax[b] = a;
-    seen_max = fmaxf(seen_max, a);
+    const float s = a;
+    const bool finite = s <= 3.402823466e38f;  // false for inf and NaN
+    nonfinite |= !finite;
+    if (finite) seen = fmaxf(seen, s);
+
+    uint32_t packed[W];
+    bool exact = !(s >= 0x1p-126f && s < 0x1p126f);
+    if (!exact) {
+      // |v| <= s and s normal: |x'| <= 1 + 2^-23, so c is within [0, 64];
+      // the clamp below only keeps the shared-memory index in range regardless
+      const float r = __frcp_rn(s);
+      float near = 1.0f;
+#pragma unroll
+      for (int i = 0; i < W; ++i) packed[i] = 0u - kPackBias;
+#pragma unroll
+      for (int j = 0; j < E; ++j) {
+        const float xp = __fmul_rn(v[j], r);
+        const float f = __fmaf_rn(xp, 32.0f, 12582944.0f);  // 1.5 * 2^23 + 32
+        const unsigned int c = min(static_cast<unsigned int>(__float_as_int(f) - 0x4B400000), 64u);
+        const float2 e = my_lut[c * 32];
+        const float d = __fsub_rn(xp, e.x);
+        near = fminf(near, fabsf(d));
+        const float step = __saturatef(__fmul_rn(d, 0x1p126f));
+        const float im = __fadd_rn(e.y, step);  // 2^23 + index
+        packed[j >> 3] += __float_as_uint(im) * (1u << (4 * (j & 7)));
+      }
+      exact = near <= kNear;
+    }
+    if (exact) {
+      // IEEE division and every threshold (a zero block gives x = 0)
+#pragma unroll
+      for (int i = 0; i < W; ++i) packed[i] = 0u;
+#pragma unroll
+      for (int j = 0; j < E; ++j) {
+        const float x = (s > 0.0f) ? __fdiv_rn(v[j], s) : 0.0f;
+        uint32_t idx = 0u;
+#pragma unroll
+        for (int k = 0; k < 15; ++k) idx += (x > tab.thr[k]) ? 1u : 0u;
+        packed[j >> 3] |= idx << (4 * (j & 7));
+      }
+    }
+    if (e0 + E <= n) {
+      if constexpr (W == 2) {
+        *reinterpret_cast<uint2*>(codes + e0 / 2) = make_uint2(packed[0], packed[1]);
+      } else {
+        *reinterpret_cast<uint4*>(codes + e0 / 2) =
+            make_uint4(packed[0], packed[1], packed[2], packed[3]);
+      }
+    } else if (e0 < n) {
+      // ragged end: bytes that hold a weight; the nibble after the last weight is 0
+#pragma unroll
+      for (int b = 0; b < E / 2; ++b) {
+        if (e0 + 2 * b >= n) break;
+        uint32_t byte = (packed[b >> 2] >> (8 * (b & 3))) & 0xffu;
+        if (e0 + 2 * b + 1 >= n) byte &= 0x0fu;
+        codes[e0 / 2 + b] = static_cast<uint8_t>(byte);
+      }
+    }
+    if ((lane & (TPB - 1)) == 0 && e0 < n) absmax[e0 / BS] = s;
+    cur = nxt;
   }
   if (nonfinite) report(st, QLORA_ERR_NONFINITE, 1u);
   // scales are >= 0, so their fp32 bit patterns order like unsigned integers
-  atomicMax(&cta_max, __float_as_uint(seen_max));
+  atomicMax(&cta_max, __float_as_uint(seen));
   __syncthreads();
   if (threadIdx.x == 0 && cta_max != 0u) atomicMax(gmax_bits, cta_max);
 }
@@ -239,20 +384,40 @@ int grid_for(int64_t work_items, int per_cta, int max_ctas) {
 }
 
 template <typename T>
-void launch_blocks(int bs, const T* w, int64_t n, const LevelTable& t, uint8_t* codes,
-                   float* absmax, unsigned int* gmax, DeviceStatus* st, cudaStream_t s) {
-  const int64_t nb = ceil_div(n, bs);
-  const int grid = grid_for(nb, 8, 148 * 16);
+qlora_status launch_blocks(int bs, const T* w, int64_t n, const LevelTable& t, uint8_t* codes,
+                           float* absmax, unsigned int* gmax, DeviceStatus* st, cudaStream_t s) {
+  CellLut cells;
+  if (!make_cell_lut(t, &cells)) return QLORA_ERR_UNSUPPORTED;
+  const int64_t chunks = ceil_div(n, bs <= 512 ? 16 : 32);
+  // persistent grid: as many CTAs as fit on the device at once
+  static int resident[2][5] = {};
+  const int ti = sizeof(T) == 4 ? 0 : 1, bi = __builtin_ctz(bs) - 6;
+  if (!resident[ti][bi]) {
+    int dev = 0, sms = 148, per_sm = 0;
+    const void* fn = bs == 64    ? reinterpret_cast<const void*>(quantize_blocks_kernel<T, 64>)
+                     : bs == 128 ? reinterpret_cast<const void*>(quantize_blocks_kernel<T, 128>)
+                     : bs == 256 ? reinterpret_cast<const void*>(quantize_blocks_kernel<T, 256>)
+                     : bs == 512 ? reinterpret_cast<const void*>(quantize_blocks_kernel<T, 512>)
+                                 : reinterpret_cast<const void*>(quantize_blocks_kernel<T, 1024>);
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, 256, 0) != cudaSuccess ||
+        per_sm < 1)
+      return QLORA_ERR_CUDA;
+    resident[ti][bi] = sms * per_sm;
+  }
+  const int grid = grid_for(chunks, 256, resident[ti][bi]);
   count_launch();
   timing_mark(QLORA_KERNEL_QUANTIZE, s, true);
   switch (bs) {
-    case 64: quantize_blocks_kernel<T, 64><<<grid, 256, 0, s>>>(w, n, t, codes, absmax, gmax, st); break;
-    case 128: quantize_blocks_kernel<T, 128><<<grid, 256, 0, s>>>(w, n, t, codes, absmax, gmax, st); break;
-    case 256: quantize_blocks_kernel<T, 256><<<grid, 256, 0, s>>>(w, n, t, codes, absmax, gmax, st); break;
-    case 512: quantize_blocks_kernel<T, 512><<<grid, 256, 0, s>>>(w, n, t, codes, absmax, gmax, st); break;
-    default: quantize_blocks_kernel<T, 1024><<<grid, 256, 0, s>>>(w, n, t, codes, absmax, gmax, st); break;
+    case 64: quantize_blocks_kernel<T, 64><<<grid, 256, 0, s>>>(w, n, t, cells, codes, absmax, gmax, st); break;
+    case 128: quantize_blocks_kernel<T, 128><<<grid, 256, 0, s>>>(w, n, t, cells, codes, absmax, gmax, st); break;
+    case 256: quantize_blocks_kernel<T, 256><<<grid, 256, 0, s>>>(w, n, t, cells, codes, absmax, gmax, st); break;
+    case 512: quantize_blocks_kernel<T, 512><<<grid, 256, 0, s>>>(w, n, t, cells, codes, absmax, gmax, st); break;
+    default: quantize_blocks_kernel<T, 1024><<<grid, 256, 0, s>>>(w, n, t, cells, codes, absmax, gmax, st); break;
   }
   timing_mark(QLORA_KERNEL_QUANTIZE, s, false);
+  return QLORA_OK;
 }
 
 }  // namespace
@@ -268,11 +433,13 @@ qlora_status launch_quantize(const void* W, int32_t w_dtype, const qlora_nf4& q,
   const int64_t n = q.rows * q.cols;
   const int64_t nb = ceil_div(n, q.blocksize);
   if (cudaMemsetAsync(ws + 256, 0, 16, s) != cudaSuccess) return QLORA_ERR_CUDA;
-  if (w_dtype == QLORA_F32)
-    launch_blocks(q.blocksize, static_cast<const float*>(W), n, t, q.codes, absmax, gmax, st, s);
-  else
-    launch_blocks(q.blocksize, static_cast<const __nv_bfloat16*>(W), n, t, q.codes, absmax, gmax,
-                  st, s);
+  const qlora_status ls =
+      (w_dtype == QLORA_F32)
+          ? launch_blocks(q.blocksize, static_cast<const float*>(W), n, t, q.codes, absmax, gmax,
+                          st, s)
+          : launch_blocks(q.blocksize, static_cast<const __nv_bfloat16*>(W), n, t, q.codes,
+                          absmax, gmax, st, s);
+  if (ls != QLORA_OK) return ls;
   if (after_launch("quantize_blocks", s) != QLORA_OK) return QLORA_ERR_CUDA;
   if (q.dq_blocksize) {
     count_launch(2);

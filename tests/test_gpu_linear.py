@@ -71,6 +71,8 @@ def test_single_linear_256():
 @pytest.mark.parametrize("M,N,K,r", [
     (1, 64, 64, 1), (3, 80, 192, 5), (17, 200, 128, 16), (130, 96, 320, 64),
     (257, 384, 256, 8), (64, 128, 4096, 256), (300, 1000, 640, 24),
+    # more 256x256 tiles than SMs with ragged edges: stream-K forward, then stream-K dX
+    (4000, 2600, 640, 16), (4000, 640, 2624, 16),
 ])
 def test_ragged_shapes(M, N, K, r):
     inp, alpha = _inputs(N, K, r, M, 1000 + M, b_std=0.05)
@@ -88,7 +90,14 @@ def test_attention_projection_4096(attn):
     shape, inp, w_hat = attn
     rows = np.sort(np.random.default_rng(0).choice(4096, 96, replace=False))
     rows = np.concatenate([[0], rows, [4095]])
-    _run(inp, shape.alpha, rows=rows, w_hat=w_hat)
+    q, Y, U, dX, dA, dB = _run(inp, shape.alpha, rows=rows, w_hat=w_hat)
+    # the same call again gives the same bits (fixed split points and summation order)
+    A, B, X, dY = (inp[k].to(DEV) for k in ("A", "B", "X", "dY"))
+    Y2 = Q.qlora_linear_fwd(q, A, B, shape.alpha, X)
+    dX2, dA2, dB2 = Q.qlora_linear_bwd(q, A, B, shape.alpha, X, U, dY)
+    torch.cuda.synchronize()
+    assert torch.equal(Y, Y2) and torch.equal(dX, dX2)
+    assert torch.equal(dA, dA2) and torch.equal(dB, dB2)
 
 
 @pytest.fixture(scope="module", params=[0, 1], ids=["gate_up", "down"])
