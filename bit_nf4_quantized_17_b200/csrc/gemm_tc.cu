@@ -29,10 +29,15 @@
 
 #include "internal.cuh"
 #include "kernels.cuh"
+#include "tc_common.cuh"
 #include "tc_ptx.cuh"
 
 namespace qlora {
 namespace {
+
+using tc::block_tables;
+using tc::expand8;
+using tc::pack_bf16x2;
 
 // warps 0-3: TMA producer, MMA issuer (and TMEM owner), two idle;
 // warps 4-19: dequantisation in two groups of 256 threads that take alternate
@@ -77,47 +82,6 @@ struct TcArgs {
   int64_t nblocks;        // entries of w.scale_codes (loads beyond it are reported)
   DeviceStatus* st;
 };
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
-
-// Expand 8 nibbles (weights k..k+7, nibble j = weight k+j) into 8 bf16 values
-// T[idx] using the byte tables L (low bytes of T[0..15]) and H (high bytes).
-__device__ __forceinline__ uint4 expand8(uint32_t x, const uint32_t (&L)[4],
-                                         const uint32_t (&H)[4]) {
-  const uint32_t sel = x & 0x77777777u;                          // byte index within a half table
-  const uint32_t msel = ((x >> 1) & 0x44444444u) | 0x32103210u;  // pick the half by bit 3
-  uint4 out;
-  {
-    const uint32_t lo = __byte_perm(__byte_perm(L[0], L[1], sel), __byte_perm(L[2], L[3], sel), msel);
-    const uint32_t hi = __byte_perm(__byte_perm(H[0], H[1], sel), __byte_perm(H[2], H[3], sel), msel);
-    out.x = __byte_perm(lo, hi, 0x5140);
-    out.y = __byte_perm(lo, hi, 0x7362);
-  }
-  {
-    const uint32_t s2 = sel >> 16, m2 = msel >> 16;
-    const uint32_t lo = __byte_perm(__byte_perm(L[0], L[1], s2), __byte_perm(L[2], L[3], s2), m2);
-    const uint32_t hi = __byte_perm(__byte_perm(H[0], H[1], s2), __byte_perm(H[2], H[3], s2), m2);
-    out.z = __byte_perm(lo, hi, 0x5140);
-    out.w = __byte_perm(lo, hi, 0x7362);
-  }
-  return out;
-}
-
-// The 16 dequantised values of one block, bf16(fp32(level[k] * s)), as byte tables.
-__device__ __forceinline__ void block_tables(const float (&lv)[16], float s, uint32_t (&L)[4],
-                                             uint32_t (&H)[4]) {
-  uint32_t P[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) P[j] = pack_bf16x2(__fmul_rn(lv[2 * j], s), __fmul_rn(lv[2 * j + 1], s));
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    L[j] = __byte_perm(P[2 * j], P[2 * j + 1], 0x6420);
-    H[j] = __byte_perm(P[2 * j], P[2 * j + 1], 0x7531);
-  }
-}
 
 __device__ __forceinline__ void store16(const TcArgs& p, int64_t row, int64_t col,
                                         const uint32_t (&r)[16]) {
@@ -544,6 +508,8 @@ __global__ void transpose_bf16_kernel(const T* __restrict__ in, int64_t rows, in
 
 // ----------------------------------------------------------------- host
 
+}  // namespace
+
 using EncodeFn = PFN_cuTensorMapEncodeTiled_v12000;
 
 EncodeFn encode_fn() {
@@ -577,6 +543,8 @@ bool make_map(CUtensorMap* map, const void* base, bool bf16, uint64_t inner, uin
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
+
+namespace {
 
 int pow2_cols(int bn) {
   int c = 32;
@@ -682,6 +650,7 @@ qlora_status launch_fused(const CUtensorMap& ma, const CUtensorMap& mb, const CU
 qlora_status tc_fused_forward(const QView& w, const LevelTable& t, const void* X, int64_t M,
                               const void* sU, const void* B, int32_t r, void* out,
                               const FusedShape& f, DeviceStatus* st, cudaStream_t s) {
+  if (tc2_eligible(M, f)) return tc2_fused_forward(w, t, X, M, sU, B, r, out, st, s);
   const int64_t N = w.rows, K = w.cols;
   const uint32_t rows = a_rows(M, f.mt);
   CUtensorMap ma, mb, ma2, mb2;
@@ -710,6 +679,7 @@ qlora_status tc_fused_forward(const QView& w, const LevelTable& t, const void* X
 qlora_status tc_fused_dgrad(const QView& w, const LevelTable& t, const void* dY, int64_t M,
                             const void* sV, const void* A, int32_t r, void* out,
                             const FusedShape& f, DeviceStatus* st, cudaStream_t s) {
+  if (tc2_eligible(M, f)) return tc2_fused_dgrad(w, t, dY, M, sV, A, r, out, st, s);
   const int64_t N = w.rows, K = w.cols;
   const uint32_t rows = a_rows(M, f.mt);
   CUtensorMap ma, mb, ma2, mb2;

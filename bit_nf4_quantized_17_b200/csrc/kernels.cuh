@@ -59,6 +59,16 @@ qlora_status tc_fused_forward(const QView& w, const LevelTable& t, const void* X
 qlora_status tc_fused_dgrad(const QView& w, const LevelTable& t, const void* dY, int64_t M,
                             const void* sV, const void* A, int32_t r, void* out,
                             const FusedShape& f, DeviceStatus* st, cudaStream_t s);
+// The same two products on CTA pairs (gemm_tc2.cu): a 512 x 256 output tile
+// per pair, each CTA dequantising half of the W tile.  Used for one split
+// with more than 256 tokens; bf16 output only.
+bool tc2_eligible(int64_t M, const FusedShape& f);
+qlora_status tc2_fused_forward(const QView& w, const LevelTable& t, const void* X, int64_t M,
+                               const void* sU, const void* B, int32_t r, void* Y,
+                               DeviceStatus* st, cudaStream_t s);
+qlora_status tc2_fused_dgrad(const QView& w, const LevelTable& t, const void* dY, int64_t M,
+                             const void* sV, const void* A, int32_t r, void* dX,
+                             DeviceStatus* st, cudaStream_t s);
 // part[z] (m_rows x n_cols fp32) = A . B^T over split z of the contraction; B has
 // b_rows rows, read as n_cols (rows past b_rows are zero).
 qlora_status tc_lora_gemm(const void* A, bool a_mn, int64_t m_rows, int64_t kdim, int64_t ld_a,
