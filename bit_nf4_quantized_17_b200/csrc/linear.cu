@@ -108,6 +108,32 @@ SmallLayout small_layout(int64_t M, int64_t N, int64_t K, int32_t r) {
 
 bool use_small(int64_t M) { return M <= kSmallM; }
 
+// A second stream for the part of the backward pass that does not feed the
+// fused dX kernel (dB, dA): launched after V is ready, it runs on the SMs that
+// kernel leaves idle in its last wave.  One per host thread and device; the
+// caller's stream waits for it before the call returns, so every call stays
+// ordered on the caller's stream (and can be captured in a CUDA graph).
+struct SideStream {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+
+qlora_status side_stream(SideStream** out) {
+  constexpr int kMaxDevices = 64;
+  thread_local SideStream per_device[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QLORA_ERR_CUDA;
+  SideStream& x = per_device[dev];
+  if (!x.stream) {
+    if (cudaEventCreateWithFlags(&x.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&x.join, cudaEventDisableTiming) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&x.stream, cudaStreamNonBlocking) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+  }
+  *out = &x;
+  return QLORA_OK;
+}
+
 ReduceArgs reduce_args(const float* part, int splits, int64_t rows, int cols, int pcols) {
   ReduceArgs a{};
   a.part = part;
@@ -298,18 +324,6 @@ qlora_status linear_backward(const qlora_nf4& W, const LevelTable& t, const void
     float* part = reinterpret_cast<float*>(ws + L.part_b);
     if (cudaMemsetAsync(sv, 0, sizeof(__nv_bfloat16) * M * 2 * span, s) != cudaSuccess)
       return QLORA_ERR_CUDA;
-    // U^T as bf16 hi (rows [0, r)) + lo (rows [r16, r16 + r)), from the saved U or X A^T
-    if (U) {
-      QLORA_TRY(transpose_to_bf16(U, true, M, r, r, ut, mp, r16, s));
-    } else {
-      QLORA_TRY(tc_lora_gemm(X, false, M, K, K, A, K, r, r16, part, sp.u, st, s));
-      ReduceArgs ra = reduce_args(part, sp.u, M, r, r16);
-      ra.o3 = ut;
-      ra.ld3 = mp;
-      ra.a3 = 1.0f;
-      ra.o3_lo = r16;
-      QLORA_TRY(splitk_reduce(ra, s));
-    }
     // B^T (r x N) so that V = dY B contracts two K-major operands
     QLORA_TRY(transpose_to_bf16(B, false, N, r, r, bt, N, 0, s));
     // V = dY B -> sV = s V as [hi | lo] and V^T as [hi ; lo]
@@ -326,42 +340,71 @@ qlora_status linear_backward(const qlora_nf4& W, const LevelTable& t, const void
       ra.o3_lo = r16;
       QLORA_TRY(splitk_reduce(ra, s));
     }
-    // dX = dY W + sV A in one kernel (split over d_out when needed)
-    if (dX) {
-      const FusedShape f = fused_shape(M, K, ceil_div(N, 64));
-      if (f.splits == 1) {
-        QLORA_TRY(tc_fused_dgrad(w, t, dY, M, sv, A, r, dX, f, st, s));
+    // dB and dA on the side stream, dX on the caller's: they share only
+    // inputs, and the side stream reuses `part` after V's reduction
+    SideStream* ss = nullptr;
+    QLORA_TRY(side_stream(&ss));
+    const cudaStream_t s2 = ss->stream;
+    if (cudaEventRecord(ss->fork, s) != cudaSuccess ||
+        cudaStreamWaitEvent(s2, ss->fork, 0) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+    auto side_work = [&]() -> qlora_status {
+      // U^T as bf16 hi (rows [0, r)) + lo (rows [r16, r16 + r)), from the saved U or X A^T
+      if (U) {
+        QLORA_TRY(transpose_to_bf16(U, true, M, r, r, ut, mp, r16, s2));
       } else {
-        float* fpart = reinterpret_cast<float*>(ws + L.fused_b);
-        QLORA_TRY(tc_fused_dgrad(w, t, dY, M, sv, A, r, fpart, f, st, s));
-        ReduceArgs rx = reduce_args(fpart, f.splits, M, static_cast<int>(K), static_cast<int>(K));
-        rx.o2 = dX;
-        rx.ld2 = K;
-        rx.a2 = 1.0f;
-        QLORA_TRY(splitk_reduce(rx, s));
+        QLORA_TRY(tc_lora_gemm(X, false, M, K, K, A, K, r, r16, part, sp.u, st, s2));
+        ReduceArgs ra = reduce_args(part, sp.u, M, r, r16);
+        ra.o3 = ut;
+        ra.ld3 = mp;
+        ra.a3 = 1.0f;
+        ra.o3_lo = r16;
+        QLORA_TRY(splitk_reduce(ra, s2));
       }
-    }
-    // dB = s dY^T U: rows d_out, contraction over tokens, hi and lo columns summed
-    QLORA_TRY(tc_lora_gemm(dY, true, N, M, N, ut, mp, 2 * r16, 2 * r16, part, sp.db, st, s));
-    {
-      ReduceArgs ra = reduce_args(part, sp.db, N, r, 2 * r16);
+      // dB = s dY^T U: rows d_out, contraction over tokens, hi and lo columns summed
+      QLORA_TRY(tc_lora_gemm(dY, true, N, M, N, ut, mp, 2 * r16, 2 * r16, part, sp.db, st, s2));
+      {
+        ReduceArgs ra = reduce_args(part, sp.db, N, r, 2 * r16);
+        ra.lo = r16;
+        ra.o1 = dB;
+        ra.ld1 = r;
+        ra.a1 = sc;
+        ra.acc1 = accumulate;
+        QLORA_TRY(splitk_reduce(ra, s2));
+      }
+      // dA = s V^T X: rows d_in, stored transposed as r x d_in
+      QLORA_TRY(tc_lora_gemm(X, true, K, M, K, vt, mp, 2 * r16, 2 * r16, part, sp.da, st, s2));
+      ReduceArgs ra = reduce_args(part, sp.da, K, r, 2 * r16);
       ra.lo = r16;
-      ra.o1 = dB;
-      ra.ld1 = r;
+      ra.o1 = dA;
+      ra.ld1 = K;
+      ra.trans1 = true;
       ra.a1 = sc;
       ra.acc1 = accumulate;
-      QLORA_TRY(splitk_reduce(ra, s));
-    }
-    // dA = s V^T X: rows d_in, stored transposed as r x d_in
-    QLORA_TRY(tc_lora_gemm(X, true, K, M, K, vt, mp, 2 * r16, 2 * r16, part, sp.da, st, s));
-    ReduceArgs ra = reduce_args(part, sp.da, K, r, 2 * r16);
-    ra.lo = r16;
-    ra.o1 = dA;
-    ra.ld1 = K;
-    ra.trans1 = true;
-    ra.a1 = sc;
-    ra.acc1 = accumulate;
-    return splitk_reduce(ra, s);
+      return splitk_reduce(ra, s2);
+    };
+    auto main_work = [&]() -> qlora_status {
+      // dX = dY W + sV A in one kernel (split over d_out when needed)
+      if (!dX) return QLORA_OK;
+      const FusedShape f = fused_shape(M, K, ceil_div(N, 64));
+      if (f.splits == 1) return tc_fused_dgrad(w, t, dY, M, sv, A, r, dX, f, st, s);
+      float* fpart = reinterpret_cast<float*>(ws + L.fused_b);
+      QLORA_TRY(tc_fused_dgrad(w, t, dY, M, sv, A, r, fpart, f, st, s));
+      ReduceArgs rx = reduce_args(fpart, f.splits, M, static_cast<int>(K), static_cast<int>(K));
+      rx.o2 = dX;
+      rx.ld2 = K;
+      rx.a2 = 1.0f;
+      return splitk_reduce(rx, s);
+    };
+    // the fused kernel is enqueued first so that its first wave takes the SMs
+    const qlora_status st_main = main_work();
+    const qlora_status st_side = side_work();
+    // join on every path, so that nothing of this call runs past it on the side stream
+    const bool joined = cudaEventRecord(ss->join, s2) == cudaSuccess &&
+                        cudaStreamWaitEvent(s, ss->join, 0) == cudaSuccess;
+    if (st_side != QLORA_OK) return st_side;
+    if (st_main != QLORA_OK) return st_main;
+    return joined ? QLORA_OK : QLORA_ERR_CUDA;
   }
   char* p = ws + kStatusBytes;
   float* u = reinterpret_cast<float*>(p);
