@@ -145,10 +145,13 @@ __device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
   return a;
 }
-// Arrive (release, cluster scope) on an mbarrier given by its shared::cluster address.
+// Arrive on an mbarrier given by its shared::cluster address (default
+// semantics).  Used after fence.proxy.async by threads whose shared-memory
+// writes the pair MMA reads: the proxy fence orders the writes for the
+// tensor core, and the arrival completes the even CTA's phase that its MMA
+// issuer waits on.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar)
-               : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
 }
 // try_wait with acquire at cluster scope (for phases completed by arrivals
 // from the other CTA of the pair).
