@@ -69,6 +69,17 @@ qlora_status tc2_fused_forward(const QView& w, const LevelTable& t, const void* 
 qlora_status tc2_fused_dgrad(const QView& w, const LevelTable& t, const void* dY, int64_t M,
                              const void* sV, const void* A, int32_t r, void* dX,
                              DeviceStatus* st, cudaStream_t s);
+// Dequant GEMVs for one or two tokens on the CUDA cores (gemv_small.cu).
+// Y = X W^T + s U B^T with U fp32 (M x r); dX partials part[c][m][k] of
+// dY W + s V A (V fp32), summed over gemv_dgrad_chunks(M, K) chunks.
+bool gemv_eligible(int64_t M, int64_t K, int32_t r);
+int gemv_dgrad_chunks(int64_t M, int64_t K);
+qlora_status gemv_forward(const QView& w, const LevelTable& t, const void* X, int64_t M,
+                          const float* U, const void* B, int32_t r, float s, void* Y,
+                          cudaStream_t st);
+qlora_status gemv_dgrad(const QView& w, const LevelTable& t, const void* dY, int64_t M,
+                        const float* V, const void* A, int32_t r, float s, float* part,
+                        cudaStream_t st);
 // part[z] (m_rows x n_cols fp32) = A . B^T over split z of the contraction; B has
 // b_rows rows, read as n_cols (rows past b_rows are zero).
 qlora_status tc_lora_gemm(const void* A, bool a_mn, int64_t m_rows, int64_t kdim, int64_t ld_a,

@@ -85,7 +85,7 @@ TcLayout tc_layout(int64_t M, int64_t N, int64_t K, int32_t r) {
 //   forward   sU [hi | lo] | U-partials | fused partials
 //   backward  sV [hi | lo] | V (fp32) | U (fp32, when recomputed) | partials | fused partials
 struct SmallLayout {
-  size_t su, part_f, fused_f, fwd_end, sv, v, u, part_b, fused_b, bwd_end;
+  size_t su, part_f, fused_f, uf, fwd_end, sv, v, u, part_b, fused_b, bwd_end;
 };
 
 SmallLayout small_layout(int64_t M, int64_t N, int64_t K, int32_t r) {
@@ -95,14 +95,18 @@ SmallLayout small_layout(int64_t M, int64_t N, int64_t K, int32_t r) {
   L.part_f = L.su + align256(2 * M * 2 * span);
   L.fused_f = L.part_f + align256(sizeof(float) * small_chunks(K) * M * r16);
   const FusedShape ff = fused_shape(M, N, K / 64);
-  L.fwd_end = L.fused_f + (ff.splits > 1 ? align256(sizeof(float) * ff.splits * M * N) : 0);
+  L.uf = L.fused_f + (ff.splits > 1 ? align256(sizeof(float) * ff.splits * M * N) : 0);
+  L.fwd_end = L.uf + align256(sizeof(float) * M * r);  // fp32 U for the GEMV path
   L.sv = kStatusBytes;
   L.v = L.sv + align256(2 * M * 2 * span);
   L.u = L.v + align256(sizeof(float) * M * r);
   L.part_b = L.u + align256(sizeof(float) * M * r);
   L.fused_b = L.part_b + align256(sizeof(float) * std::max(small_chunks(K), small_chunks(N)) * M * r16);
   const FusedShape fb = fused_shape(M, K, ceil_div(N, 64));
-  L.bwd_end = L.fused_b + (fb.splits > 1 ? align256(sizeof(float) * fb.splits * M * K) : 0);
+  const size_t fused_parts = fb.splits > 1 ? sizeof(float) * fb.splits * M * K : 0;
+  const size_t gemv_parts =
+      gemv_eligible(M, K, r) ? sizeof(float) * gemv_dgrad_chunks(M, K) * M * K : 0;
+  L.bwd_end = L.fused_b + align256(std::max(fused_parts, gemv_parts));
   return L;
 }
 
@@ -185,6 +189,17 @@ qlora_status linear_forward(const qlora_nf4& W, const LevelTable& t, const void*
     const int32_t r16 = lora_rows(r), span = lora_span(r);
     char* su = ws + L.su;
     float* part = reinterpret_cast<float*>(ws + L.part_f);
+    if (gemv_eligible(M, K, r)) {
+      // one or two tokens: U = X A^T in fp32, then the dequant GEMV adds s U B^T itself
+      float* u = U_save ? U_save : reinterpret_cast<float*>(ws + L.uf);
+      QLORA_TRY(small_down_partial(X, A, static_cast<int>(M), K, r, part, s));
+      ReduceArgs ra = reduce_args(part, small_chunks(K), M, r, r16);
+      ra.o1 = u;
+      ra.ld1 = r;
+      ra.a1 = 1.0f;
+      QLORA_TRY(splitk_reduce(ra, s));
+      return gemv_forward(w, t, X, M, u, B, r, sc, Y, s);
+    }
     if (cudaMemsetAsync(su, 0, sizeof(__nv_bfloat16) * M * 2 * span, s) != cudaSuccess)
       return QLORA_ERR_CUDA;
     QLORA_TRY(small_down_partial(X, A, static_cast<int>(M), K, r, part, s));
@@ -270,19 +285,22 @@ qlora_status linear_backward(const qlora_nf4& W, const LevelTable& t, const void
     char* sv = ws + L.sv;
     float* v = reinterpret_cast<float*>(ws + L.v);
     float* part = reinterpret_cast<float*>(ws + L.part_b);
-    if (cudaMemsetAsync(sv, 0, sizeof(__nv_bfloat16) * M * 2 * span, s) != cudaSuccess)
+    const bool gemv = gemv_eligible(M, K, r);
+    if (!gemv && cudaMemsetAsync(sv, 0, sizeof(__nv_bfloat16) * M * 2 * span, s) != cudaSuccess)
       return QLORA_ERR_CUDA;
-    // V = dY B -> V (fp32) and sV = s V as [hi | lo]
+    // V = dY B -> V (fp32) and, for the tensor-core kernel, sV = s V as [hi | lo]
     QLORA_TRY(small_v_partial(dY, B, m, N, r, part, s));
     {
       ReduceArgs ra = reduce_args(part, small_chunks(N), M, r, r16);
       ra.o1 = v;
       ra.ld1 = r;
       ra.a1 = 1.0f;
-      ra.o2 = sv;
-      ra.ld2 = 2 * span;
-      ra.a2 = sc;
-      ra.o2_lo = span;
+      if (!gemv) {
+        ra.o2 = sv;
+        ra.ld2 = 2 * span;
+        ra.a2 = sc;
+        ra.o2_lo = span;
+      }
       QLORA_TRY(splitk_reduce(ra, s));
     }
     if (!U) {
@@ -295,7 +313,17 @@ qlora_status linear_backward(const qlora_nf4& W, const LevelTable& t, const void
       QLORA_TRY(splitk_reduce(ra, s));
       U = u;
     }
-    if (dX) {
+    if (dX && gemv) {
+      // dX = dY W + s V A: CTA partials of the dequant GEMV, summed in order
+      float* fpart = reinterpret_cast<float*>(ws + L.fused_b);
+      QLORA_TRY(gemv_dgrad(w, t, dY, M, v, A, r, sc, fpart, s));
+      ReduceArgs rx = reduce_args(fpart, gemv_dgrad_chunks(M, K), M, static_cast<int>(K),
+                                  static_cast<int>(K));
+      rx.o2 = dX;
+      rx.ld2 = K;
+      rx.a2 = 1.0f;
+      QLORA_TRY(splitk_reduce(rx, s));
+    } else if (dX) {
       const FusedShape f = fused_shape(M, K, ceil_div(N, 64));
       if (f.splits == 1) {
         QLORA_TRY(tc_fused_dgrad(w, t, dY, M, sv, A, r, dX, f, st, s));

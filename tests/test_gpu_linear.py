@@ -71,8 +71,10 @@ def test_single_linear_256():
 @pytest.mark.parametrize("M,N,K,r", [
     (1, 64, 64, 1), (3, 80, 192, 5), (17, 200, 128, 16), (130, 96, 320, 64),
     (257, 384, 256, 8), (64, 128, 4096, 256), (300, 1000, 640, 24),
-    # more 256x256 tiles than SMs with ragged edges: stream-K forward, then stream-K dX
+    # more output tiles than SMs, ragged edges (CTA-pair kernels)
     (4000, 2600, 640, 16), (4000, 640, 2624, 16),
+    # two tokens (dequant GEMVs): K below one 1024-column group, and a ragged second group
+    (2, 200, 320, 16), (2, 4104, 1088, 24),
 ])
 def test_ragged_shapes(M, N, K, r):
     inp, alpha = _inputs(N, K, r, M, 1000 + M, b_std=0.05)
