@@ -435,22 +435,45 @@ __device__ __forceinline__ void reduce_store(float v, int64_t i, int j, float* o
   }
 }
 
+// With o2_pad the padding columns of o2 ([cols, o2_lo) and [o2_lo + cols,
+// 2 o2_lo) of every row) are written as zeros too, so o2 needs no memset.
 __global__ void splitk_reduce_kernel(const float* __restrict__ part, int splits, int64_t rows,
                                      int cols, int pcols, int lo, float* o1, int64_t ld1,
                                      int trans1, float a1, int acc1, __nv_bfloat16* o2, int64_t ld2,
                                      float a2, int o2_lo, __nv_bfloat16* o3, int64_t ld3, float a3,
-                                     int o3_lo) {
+                                     int o3_lo, int o2_pad) {
   const int64_t total = rows * cols;
+  const int pad = (o2 && o2_pad) ? o2_lo - cols : 0;
+  const int64_t total_pad = rows * 2 * pad;
   const int64_t split_stride = rows * pcols;
-  for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
-       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+  for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+       e < total + total_pad; e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    if (e >= total) {
+      const int64_t p = e - total;
+      const int64_t i = p / (2 * pad);
+      const int c = static_cast<int>(p - i * 2 * pad);
+      o2[i * ld2 + ((c < pad) ? cols + c : o2_lo + cols + (c - pad))] = __float2bfloat16_rn(0.0f);
+      continue;
+    }
     const int64_t i = e / cols;
     const int j = static_cast<int>(e - i * cols);
     const float* src = part + i * pcols + j;
+    // up to 8 splits are loaded together, then added in split order
     float v = 0.0f;
-    for (int z = 0; z < splits; ++z) {
-      v += src[z * split_stride];
-      if (lo) v += src[z * split_stride + lo];
+    for (int z0 = 0; z0 < splits; z0 += 8) {
+      float h[8], l[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        h[u] = (z0 + u < splits) ? src[(z0 + u) * split_stride] : 0.0f;
+        l[u] = (lo && z0 + u < splits) ? src[(z0 + u) * split_stride + lo] : 0.0f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (z0 + u < splits) {
+          v += h[u];
+          if (lo) v += l[u];
+        }
+      }
     }
     reduce_store(v, i, j, o1, ld1, trans1, a1, acc1, o2, ld2, a2, o2_lo, o3, ld3, a3, o3_lo);
   }
@@ -463,10 +486,20 @@ __global__ void splitk_reduce_warp_kernel(const float* __restrict__ part, int sp
                                           int cols, int pcols, int lo, float* o1, int64_t ld1,
                                           int trans1, float a1, int acc1, __nv_bfloat16* o2,
                                           int64_t ld2, float a2, int o2_lo, __nv_bfloat16* o3,
-                                          int64_t ld3, float a3, int o3_lo) {
+                                          int64_t ld3, float a3, int o3_lo, int o2_pad) {
   const int64_t total = rows * cols;
   const int64_t split_stride = rows * pcols;
   const int lane = threadIdx.x & 31;
+  if (o2 && o2_pad) {
+    // the padding columns of o2, one thread each
+    const int pad = o2_lo - cols;
+    for (int64_t p = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+         p < rows * 2 * pad; p += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+      const int64_t i = p / (2 * pad);
+      const int c = static_cast<int>(p - i * 2 * pad);
+      o2[i * ld2 + ((c < pad) ? cols + c : o2_lo + cols + (c - pad))] = __float2bfloat16_rn(0.0f);
+    }
+  }
   for (int64_t e = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; e < total;
        e += (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5) {
     const int64_t i = e / cols;
@@ -743,13 +776,15 @@ qlora_status splitk_reduce(const ReduceArgs& a, cudaStream_t s) {
     splitk_reduce_warp_kernel<<<grid, 256, 0, s>>>(
         a.part, a.splits, a.rows, a.cols, a.pcols, a.lo, a.o1, a.ld1, a.trans1 ? 1 : 0, a.a1,
         a.acc1 ? 1 : 0, static_cast<__nv_bfloat16*>(a.o2), a.ld2, a.a2, a.o2_lo,
-        static_cast<__nv_bfloat16*>(a.o3), a.ld3, a.a3, a.o3_lo);
+        static_cast<__nv_bfloat16*>(a.o3), a.ld3, a.a3, a.o3_lo, a.o2_pad);
   } else {
-    const int grid = static_cast<int>(std::min<int64_t>(ceil_div(total, 256), 148 * 8));
+    const int64_t pad_items = (a.o2 && a.o2_pad) ? a.rows * 2 * (a.o2_lo - a.cols) : 0;
+    const int grid =
+        static_cast<int>(std::min<int64_t>(ceil_div(total + pad_items, 256), 148 * 8));
     splitk_reduce_kernel<<<grid, 256, 0, s>>>(
         a.part, a.splits, a.rows, a.cols, a.pcols, a.lo, a.o1, a.ld1, a.trans1 ? 1 : 0, a.a1,
         a.acc1 ? 1 : 0, static_cast<__nv_bfloat16*>(a.o2), a.ld2, a.a2, a.o2_lo,
-        static_cast<__nv_bfloat16*>(a.o3), a.ld3, a.a3, a.o3_lo);
+        static_cast<__nv_bfloat16*>(a.o3), a.ld3, a.a3, a.o3_lo, a.o2_pad);
   }
   return after_launch("splitk_reduce", s);
 }

@@ -104,6 +104,7 @@ struct ReduceArgs {
   int64_t ld3;
   float a3;
   int o3_lo;
+  int o2_pad;  // > 0: also write zeros to o2 columns [cols, o2_lo) and [o2_lo + cols, 2 o2_lo)
 };
 qlora_status splitk_reduce(const ReduceArgs& a, cudaStream_t s);
 qlora_status transpose_to_bf16(const void* in, bool in_f32, int64_t rows, int cols, int64_t ld_in,

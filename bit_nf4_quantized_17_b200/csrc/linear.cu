@@ -200,8 +200,6 @@ qlora_status linear_forward(const qlora_nf4& W, const LevelTable& t, const void*
       QLORA_TRY(splitk_reduce(ra, s));
       return gemv_forward(w, t, X, M, u, B, r, sc, Y, s);
     }
-    if (cudaMemsetAsync(su, 0, sizeof(__nv_bfloat16) * M * 2 * span, s) != cudaSuccess)
-      return QLORA_ERR_CUDA;
     QLORA_TRY(small_down_partial(X, A, static_cast<int>(M), K, r, part, s));
     ReduceArgs ra = reduce_args(part, small_chunks(K), M, r, r16);
     ra.o1 = U_save;
@@ -211,6 +209,7 @@ qlora_status linear_forward(const qlora_nf4& W, const LevelTable& t, const void*
     ra.ld2 = 2 * span;
     ra.a2 = sc;
     ra.o2_lo = span;
+    ra.o2_pad = 1;  // the padding columns meet zero B columns in the MMA: written as zeros
     QLORA_TRY(splitk_reduce(ra, s));
     const FusedShape f = fused_shape(M, N, K / 64);
     if (f.splits == 1) return tc_fused_forward(w, t, X, M, su, B, r, Y, f, st, s);
@@ -228,9 +227,6 @@ qlora_status linear_forward(const qlora_nf4& W, const LevelTable& t, const void*
     const int32_t r16 = lora_rows(r), span = lora_span(r);
     char* su = ws + L.su;
     float* part = reinterpret_cast<float*>(ws + L.part_f);
-    // the padding columns of [hi | lo] meet zero B columns in the MMA: keep them zero
-    if (cudaMemsetAsync(su, 0, sizeof(__nv_bfloat16) * M * 2 * span, s) != cudaSuccess)
-      return QLORA_ERR_CUDA;
     // U = X A^T (split-K over d_in) -> U_save (fp32) and sU = s U as bf16 hi + lo
     QLORA_TRY(tc_lora_gemm(X, false, M, K, K, A, K, r, r16, part, sp.u, st, s));
     ReduceArgs ra = reduce_args(part, sp.u, M, r, r16);
@@ -241,6 +237,7 @@ qlora_status linear_forward(const qlora_nf4& W, const LevelTable& t, const void*
     ra.ld2 = 2 * span;
     ra.a2 = sc;
     ra.o2_lo = span;
+    ra.o2_pad = 1;  // the padding columns meet zero B columns in the MMA: written as zeros
     QLORA_TRY(splitk_reduce(ra, s));
     // Y = X W^T + sU B^T in one kernel (split over d_in, then summed, when the
     // output alone would leave SMs idle)
@@ -286,8 +283,6 @@ qlora_status linear_backward(const qlora_nf4& W, const LevelTable& t, const void
     float* v = reinterpret_cast<float*>(ws + L.v);
     float* part = reinterpret_cast<float*>(ws + L.part_b);
     const bool gemv = gemv_eligible(M, K, r);
-    if (!gemv && cudaMemsetAsync(sv, 0, sizeof(__nv_bfloat16) * M * 2 * span, s) != cudaSuccess)
-      return QLORA_ERR_CUDA;
     // V = dY B -> V (fp32) and, for the tensor-core kernel, sV = s V as [hi | lo]
     QLORA_TRY(small_v_partial(dY, B, m, N, r, part, s));
     {
@@ -300,6 +295,7 @@ qlora_status linear_backward(const qlora_nf4& W, const LevelTable& t, const void
         ra.ld2 = 2 * span;
         ra.a2 = sc;
         ra.o2_lo = span;
+        ra.o2_pad = 1;
       }
       QLORA_TRY(splitk_reduce(ra, s));
     }
@@ -350,8 +346,6 @@ qlora_status linear_backward(const qlora_nf4& W, const LevelTable& t, const void
     char* sv = ws + L.sv;
     char* vt = ws + L.vt;
     float* part = reinterpret_cast<float*>(ws + L.part_b);
-    if (cudaMemsetAsync(sv, 0, sizeof(__nv_bfloat16) * M * 2 * span, s) != cudaSuccess)
-      return QLORA_ERR_CUDA;
     // B^T (r x N) so that V = dY B contracts two K-major operands
     QLORA_TRY(transpose_to_bf16(B, false, N, r, r, bt, N, 0, s));
     // V = dY B -> sV = s V as [hi | lo] and V^T as [hi ; lo]
@@ -362,6 +356,7 @@ qlora_status linear_backward(const qlora_nf4& W, const LevelTable& t, const void
       ra.ld2 = 2 * span;
       ra.a2 = sc;
       ra.o2_lo = span;
+      ra.o2_pad = 1;
       ra.o3 = vt;
       ra.ld3 = mp;
       ra.a3 = 1.0f;
