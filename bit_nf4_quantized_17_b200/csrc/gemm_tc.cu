@@ -633,8 +633,10 @@ uint32_t a_rows(int64_t M, int mt) {
   return static_cast<uint32_t>(r16 < full ? r16 : full);
 }
 
+// Splits of a rank-r GEMM: as many as keep the grid within one wave (two
+// CTAs per SM), and at least four k-tiles per split.
 int tc_split_count(int64_t m_tiles, int64_t k_tiles) {
-  int64_t s = (2 * 148 + m_tiles - 1) / m_tiles;
+  int64_t s = (2 * 148) / m_tiles;
   const int64_t max_s = k_tiles / 4 > 0 ? k_tiles / 4 : 1;
   if (s > max_s) s = max_s;
   if (s < 1) s = 1;

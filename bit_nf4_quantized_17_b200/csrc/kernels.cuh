@@ -69,14 +69,18 @@ qlora_status tc2_fused_forward(const QView& w, const LevelTable& t, const void* 
 qlora_status tc2_fused_dgrad(const QView& w, const LevelTable& t, const void* dY, int64_t M,
                              const void* sV, const void* A, int32_t r, void* dX,
                              DeviceStatus* st, cudaStream_t s);
-// Dequant GEMVs for one or two tokens on the CUDA cores (gemv_small.cu).
-// Y = X W^T + s U B^T with U fp32 (M x r); dX partials part[c][m][k] of
-// dY W + s V A (V fp32), summed over gemv_dgrad_chunks(M, K) chunks.
+// Forward for M <= 16 tokens with the dequantised W in TMEM as the MMA's A
+// operand (gemm_tc_decode.cu): Y^T = W X^T + B (sU)^T; with splits > 1 `out`
+// receives fp32 partials out[z] of M x N, summed by splitk_reduce.
+int tc_decode_splits(int64_t M, int64_t N, int64_t K);
+qlora_status tc_decode_forward(const QView& w, const LevelTable& t, const void* X, int64_t M,
+                               const void* sU, const void* B, int32_t r, void* out, int splits,
+                               DeviceStatus* st, cudaStream_t s);
+// Dequant GEMV for the dX product of one or two tokens on the CUDA cores
+// (gemv_small.cu): partials part[c][m][k] of dY W + s V A (V fp32), summed
+// over gemv_dgrad_chunks(M, K) chunks.
 bool gemv_eligible(int64_t M, int64_t K, int32_t r);
 int gemv_dgrad_chunks(int64_t M, int64_t K);
-qlora_status gemv_forward(const QView& w, const LevelTable& t, const void* X, int64_t M,
-                          const float* U, const void* B, int32_t r, float s, void* Y,
-                          cudaStream_t st);
 qlora_status gemv_dgrad(const QView& w, const LevelTable& t, const void* dY, int64_t M,
                         const float* V, const void* A, int32_t r, float s, float* part,
                         cudaStream_t st);

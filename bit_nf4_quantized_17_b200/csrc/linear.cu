@@ -85,7 +85,7 @@ TcLayout tc_layout(int64_t M, int64_t N, int64_t K, int32_t r) {
 //   forward   sU [hi | lo] | U-partials | fused partials
 //   backward  sV [hi | lo] | V (fp32) | U (fp32, when recomputed) | partials | fused partials
 struct SmallLayout {
-  size_t su, part_f, fused_f, uf, fwd_end, sv, v, u, part_b, fused_b, bwd_end;
+  size_t su, part_f, fused_f, fwd_end, sv, v, u, part_b, fused_b, bwd_end;
 };
 
 SmallLayout small_layout(int64_t M, int64_t N, int64_t K, int32_t r) {
@@ -95,8 +95,8 @@ SmallLayout small_layout(int64_t M, int64_t N, int64_t K, int32_t r) {
   L.part_f = L.su + align256(2 * M * 2 * span);
   L.fused_f = L.part_f + align256(sizeof(float) * small_chunks(K) * M * r16);
   const FusedShape ff = fused_shape(M, N, K / 64);
-  L.uf = L.fused_f + (ff.splits > 1 ? align256(sizeof(float) * ff.splits * M * N) : 0);
-  L.fwd_end = L.uf + align256(sizeof(float) * M * r);  // fp32 U for the GEMV path
+  const int fsplits = std::max(ff.splits, tc_decode_splits(M, N, K));
+  L.fwd_end = L.fused_f + (fsplits > 1 ? align256(sizeof(float) * fsplits * M * N) : 0);
   L.sv = kStatusBytes;
   L.v = L.sv + align256(2 * M * 2 * span);
   L.u = L.v + align256(sizeof(float) * M * r);
@@ -189,17 +189,6 @@ qlora_status linear_forward(const qlora_nf4& W, const LevelTable& t, const void*
     const int32_t r16 = lora_rows(r), span = lora_span(r);
     char* su = ws + L.su;
     float* part = reinterpret_cast<float*>(ws + L.part_f);
-    if (gemv_eligible(M, K, r)) {
-      // one or two tokens: U = X A^T in fp32, then the dequant GEMV adds s U B^T itself
-      float* u = U_save ? U_save : reinterpret_cast<float*>(ws + L.uf);
-      QLORA_TRY(small_down_partial(X, A, static_cast<int>(M), K, r, part, s));
-      ReduceArgs ra = reduce_args(part, small_chunks(K), M, r, r16);
-      ra.o1 = u;
-      ra.ld1 = r;
-      ra.a1 = 1.0f;
-      QLORA_TRY(splitk_reduce(ra, s));
-      return gemv_forward(w, t, X, M, u, B, r, sc, Y, s);
-    }
     QLORA_TRY(small_down_partial(X, A, static_cast<int>(M), K, r, part, s));
     ReduceArgs ra = reduce_args(part, small_chunks(K), M, r, r16);
     ra.o1 = U_save;
@@ -211,11 +200,12 @@ qlora_status linear_forward(const qlora_nf4& W, const LevelTable& t, const void*
     ra.o2_lo = span;
     ra.o2_pad = 1;  // the padding columns meet zero B columns in the MMA: written as zeros
     QLORA_TRY(splitk_reduce(ra, s));
-    const FusedShape f = fused_shape(M, N, K / 64);
-    if (f.splits == 1) return tc_fused_forward(w, t, X, M, su, B, r, Y, f, st, s);
+    // Y = X W^T + sU B^T with W in TMEM as the MMA's A operand
+    const int splits = tc_decode_splits(M, N, K);
+    if (splits == 1) return tc_decode_forward(w, t, X, M, su, B, r, Y, 1, st, s);
     float* fpart = reinterpret_cast<float*>(ws + L.fused_f);
-    QLORA_TRY(tc_fused_forward(w, t, X, M, su, B, r, fpart, f, st, s));
-    ReduceArgs ry = reduce_args(fpart, f.splits, M, static_cast<int>(N), static_cast<int>(N));
+    QLORA_TRY(tc_decode_forward(w, t, X, M, su, B, r, fpart, splits, st, s));
+    ReduceArgs ry = reduce_args(fpart, splits, M, static_cast<int>(N), static_cast<int>(N));
     ry.o2 = Y;
     ry.ld2 = N;
     ry.a2 = 1.0f;
