@@ -294,6 +294,28 @@ def time_decode(Q, WL, dev, peaks, steps=30, warmup=5):
     return out
 
 
+def time_merge(Q, sets, shape, peaks, steps=20):
+    """qlora_merge of the bench's quantised weights into bf16 (the deployment
+    step after training): NF4 bytes + A + B read, 2 bytes per weight written."""
+    N, K, r = shape.d_out, shape.d_in, shape.r
+    outs = [torch.empty((N, K), dtype=torch.bfloat16, device=s.A.device) for s in sets]
+    for i in range(3):
+        Q.qlora_merge(sets[i % N_SETS].q, sets[i % N_SETS].A, sets[i % N_SETS].B, shape.alpha,
+                      out=outs[i % N_SETS])
+    torch.cuda.synchronize()
+    Q.qlora_timing_begin((Q.QLORA_KERNEL_MERGE,), max_launches=steps)
+    for i in range(steps):
+        s = sets[i % N_SETS]
+        Q.qlora_merge(s.q, s.A, s.B, shape.alpha, out=outs[i % N_SETS])
+    torch.cuda.synchronize()
+    ms, n = Q.qlora_timing_end()[Q.QLORA_KERNEL_MERGE]
+    t = ms * 1e-3 / max(n, 1)
+    nbytes = nf4_bytes(N, K) + 2 * r * (N + K) + 2 * N * K
+    return {"us": round(t * 1e6, 2), "gbs": round(nbytes / t / 1e9, 1),
+            "frac_hbm": round(nbytes / t / 1e9 / peaks["hbm"], 4),
+            "workload": f"{N}x{K} r={r}: NF4 + A + B read, bf16 W written; {n} launches"}
+
+
 def cpu_oracle_sample(shape, tokens_sample, WL, min_seconds=10.0, max_repeats=20):
     """Oracle quantise of the full W + fwd/bwd on `tokens_sample` tokens,
     repeated until about `min_seconds` of CPU work (at least 3 repeats)."""
@@ -428,6 +450,9 @@ def run_ours(args):
     decode = None
     if rank == 0 and world == 1 and not args.no_decode:
         decode = time_decode(Q, WL, dev, peaks)
+    merge = None
+    if rank == 0 and world == 1 and not args.no_decode:
+        merge = time_merge(Q, sets, shape, peaks)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -451,7 +476,7 @@ def run_ours(args):
         "bwd_tflops": round((fwd_bwd_flops(M, N, K, r) - fwd_flops(M, N, K, r)) / t_bwd / 1e12, 2),
         "frac_of_bf16_peak": round(value / world / peaks["bf16_sustained"], 4),
         "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
-        "gpu_launches": launches, "clocks": clk.summary(), "decode": decode,
+        "gpu_launches": launches, "clocks": clk.summary(), "decode": decode, "merge": merge,
         "peaks": peaks,
     }
     print(json.dumps(line), flush=True)

@@ -178,6 +178,20 @@ qlora_status qlora_dequantize(const qlora_nf4* q, void* W_out, int32_t out_dtype
   return launch_dequantize(*q, *t, W_out, out_dtype, static_cast<cudaStream_t>(stream));
 }
 
+qlora_status qlora_merge(const qlora_nf4* W, const void* A, const void* B, int32_t r,
+                         float alpha, void* W_out, void* stream) {
+  if (!W || !A || !B || !W_out) return QLORA_ERR_NULL;
+  qlora_status st = check_nf4_shape(*W);
+  if (st != QLORA_OK) return st;
+  if ((st = check_nf4_ptrs(*W)) != QLORA_OK) return st;
+  if (W->cols % W->blocksize != 0) return QLORA_ERR_UNSUPPORTED;
+  if (r < 1 || r > 256) return QLORA_ERR_SHAPE;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(W_out)) return QLORA_ERR_ALIGN;
+  const LevelTable* t = level_table(W->table);
+  if (!t) return QLORA_ERR_UNSUPPORTED;
+  return launch_merge(*W, *t, A, B, r, alpha, W_out, static_cast<cudaStream_t>(stream));
+}
+
 qlora_status qlora_linear_workspace(int64_t M, int64_t N, int64_t K, int32_t r, size_t* fwd_bytes,
                                     size_t* bwd_bytes) {
   if (M < 0 || N < 1 || K < 1 || r < 1 || r > 256) return QLORA_ERR_SHAPE;
@@ -194,7 +208,8 @@ static qlora_status check_linear(const qlora_nf4* W, const void* A, const void* 
   qlora_status st = check_nf4_shape(*W);
   if (st != QLORA_OK) return st;
   if ((st = check_nf4_ptrs(*W)) != QLORA_OK) return st;
-  if (W->blocksize != 64 || W->cols % 64 != 0) return QLORA_ERR_UNSUPPORTED;
+  // blocks never straddle rows, so every 64-weight k-tile lies in one block
+  if (W->cols % W->blocksize != 0) return QLORA_ERR_UNSUPPORTED;
   if (r < 1 || r > 256 || M < 0) return QLORA_ERR_SHAPE;
   if (!aligned16(A) || !aligned16(B) || !aligned16(X) || !aligned16(workspace))
     return QLORA_ERR_ALIGN;  // (a NULL X with M = 0 counts as aligned)

@@ -38,7 +38,7 @@ __device__ __forceinline__ float load_operand(const Operand& o, int64_t i, int64
     const uint8_t byte = __ldg(o.w.codes + (e >> 1));
     const int idx = (e & 1) ? (byte >> 4) : (byte & 15);
     // the product uses the dequantised weight rounded to bf16
-    return __bfloat162float(__float2bfloat16_rn(__fmul_rn(lv[idx], block_scale(o.w, e >> 6, mu))));
+    return __bfloat162float(__float2bfloat16_rn(__fmul_rn(lv[idx], block_scale(o.w, e >> (6 + o.w.bs_shift), mu))));
   }
 }
 

@@ -309,7 +309,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                                                : static_cast<int64_t>(kg) * 64 + row;
         const int64_t kb = (BMODE == B_DQ_K) ? kg : (n0 / 64 + q);
         if (wrow >= p.w.rows || kb >= p.kblocks) return RawScale{0.0f, 0.0f, false};
-        const int64_t b = wrow * p.kblocks + kb;
+        const int64_t b = wrow * (p.kblocks >> p.w.bs_shift) + (kb >> p.w.bs_shift);
         if (b >= p.nblocks) {
           report(p.st, QLORA_ERR_SHAPE, 201u);
           return RawScale{0.0f, 0.0f, false};
@@ -702,7 +702,7 @@ qlora_status tc_fused_forward(const QView& w, const LevelTable& t, const void* X
   p.k2_last_steps = ((r - 64 * (p.k2_half - 1)) + 15) / 16;
   p.w = w;
   p.kblocks = static_cast<int>(K / 64);
-  p.nblocks = N * K / 64;
+  p.nblocks = (N * K / 64) >> w.bs_shift;
   p.out = out;
   p.ldo = N;
   p.out_bf16 = f.splits == 1 ? 1 : 0;
@@ -731,7 +731,7 @@ qlora_status tc_fused_dgrad(const QView& w, const LevelTable& t, const void* dY,
   p.b2_mn = 1;
   p.w = w;
   p.kblocks = static_cast<int>(K / 64);
-  p.nblocks = N * K / 64;
+  p.nblocks = (N * K / 64) >> w.bs_shift;
   p.out = out;
   p.ldo = K;
   p.out_bf16 = f.splits == 1 ? 1 : 0;

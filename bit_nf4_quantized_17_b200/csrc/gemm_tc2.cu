@@ -252,7 +252,7 @@ tc2_fused_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                                              : static_cast<int64_t>(kt) * 64 + row;
       const int64_t kb = (BMODE == B_DQ_K) ? kt : (nh / 64 + q);
       if (wrow >= p.w.rows || kb >= p.kblocks) return RawScale{0.0f, 0.0f, false};
-      const int64_t b = wrow * p.kblocks + kb;
+      const int64_t b = wrow * (p.kblocks >> p.w.bs_shift) + (kb >> p.w.bs_shift);
       if (b >= p.nblocks) {
         report(p.st, QLORA_ERR_SHAPE, 211u);
         return RawScale{0.0f, 0.0f, false};
@@ -371,7 +371,7 @@ Tc2Args args_of(const QView& w, int64_t M, int64_t n_out, int32_t r, void* out, 
   p.a_bytes = kABytes;
   p.w = w;
   p.kblocks = static_cast<int32_t>(w.cols / 64);
-  p.nblocks = w.rows * w.cols / 64;
+  p.nblocks = (w.rows * w.cols / 64) >> w.bs_shift;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.ldo = n_out;
   p.out_elems = M * n_out;

@@ -214,7 +214,7 @@ tc_decode_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
     };
     auto load_scale = [&](int i) -> RawScale {
       if (i >= kn || wrow >= p.w.rows) return RawScale{0.0f, 0.0f, false};
-      const int64_t b = wrow * p.kblocks + kt0 + i;
+      const int64_t b = wrow * (p.kblocks >> p.w.bs_shift) + ((kt0 + i) >> p.w.bs_shift);
       if (b >= p.nblocks) {
         report(p.st, QLORA_ERR_SHAPE, 221u);
         return RawScale{0.0f, 0.0f, false};
@@ -331,7 +331,7 @@ qlora_status tc_decode_forward(const QView& w, const LevelTable& t, const void* 
   p.k2_last_steps = ((r - 64 * (p.k2_half - 1)) + 15) / 16;
   p.w = w;
   p.kblocks = static_cast<int32_t>(K / 64);
-  p.nblocks = N * K / 64;
+  p.nblocks = (N * K / 64) >> w.bs_shift;
   p.out = out;
   p.out_bf16 = splits == 1 ? 1 : 0;
   p.split_stride = M * N;

@@ -39,7 +39,7 @@ gemv_dgrad_kernel(QView w, LevelTable tab, const __nv_bfloat16* __restrict__ dY,
                   int n_kgroups, float* __restrict__ part) {
   extern __shared__ float red[];  // kWarps * MM * kRedStride fp32
   const int64_t N = w.rows;
-  const int K = static_cast<int>(w.cols), nb = K / 64;
+  const int K = static_cast<int>(w.cols), nb = K >> (6 + w.bs_shift);  // blocks per row
   const int g = blockIdx.x % n_kgroups;
   const int c = blockIdx.x / n_kgroups;
   const int C = gridDim.x / n_kgroups;
@@ -47,7 +47,7 @@ gemv_dgrad_kernel(QView w, LevelTable tab, const __nv_bfloat16* __restrict__ dY,
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int k0 = 1024 * g + 32 * lane;
   const bool active = k0 < K;
-  const int b = k0 >> 6;
+  const int b = k0 >> (6 + w.bs_shift);  // this lane's block within the row
   float lv[16];
 #pragma unroll
   for (int j = 0; j < 16; ++j) lv[j] = tab.level[j];

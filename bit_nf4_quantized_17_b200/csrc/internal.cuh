@@ -60,6 +60,10 @@ qlora_status launch_quantize(const void* W, int32_t w_dtype, const qlora_nf4& q,
 qlora_status launch_dequantize(const qlora_nf4& q, const LevelTable& t, void* out,
                                int32_t out_dtype, cudaStream_t s);
 
+// merge.cu: W_out = bf16(dequant(W) + (alpha / r) B A)
+qlora_status launch_merge(const qlora_nf4& q, const LevelTable& t, const void* A, const void* B,
+                          int32_t r, float alpha, void* out, cudaStream_t s);
+
 // Everything a linear-layer kernel needs to read a quantised W.
 struct QView {
   const uint8_t* codes;
@@ -68,6 +72,7 @@ struct QView {
   const float* mean;
   int64_t rows, cols;
   int32_t dq_shift;  // log2(dq_blocksize); -1 without double quantisation
+  int32_t bs_shift;  // log2(blocksize / 64): 64-weight k-tile t of a row lies in block t >> bs_shift
 };
 
 #ifdef __CUDACC__

@@ -26,7 +26,8 @@ size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
 
 QView view_of(const qlora_nf4& W) {
   return QView{W.codes, W.scale_codes, W.factors, W.mean, W.rows, W.cols,
-               W.dq_blocksize ? __builtin_ctz(W.dq_blocksize) : -1};
+               W.dq_blocksize ? __builtin_ctz(W.dq_blocksize) : -1,
+               __builtin_ctz(W.blocksize) - 6};
 }
 
 float lora_scale(float alpha, int32_t r) { return alpha / static_cast<float>(r); }

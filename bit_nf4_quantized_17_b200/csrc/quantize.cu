@@ -456,7 +456,7 @@ qlora_status launch_quantize(const void* W, int32_t w_dtype, const qlora_nf4& q,
 qlora_status launch_dequantize(const qlora_nf4& q, const LevelTable& t, void* out,
                                int32_t out_dtype, cudaStream_t s) {
   QView w{q.codes, q.scale_codes, q.factors, q.mean, q.rows, q.cols,
-          q.dq_blocksize ? __builtin_ctz(q.dq_blocksize) : -1};
+          q.dq_blocksize ? __builtin_ctz(q.dq_blocksize) : -1, __builtin_ctz(q.blocksize) - 6};
   const int bs_shift = __builtin_ctz(q.blocksize);
   const int64_t n = q.rows * q.cols;
   const int grid = grid_for(ceil_div(n, 8), 256, 148 * 8);

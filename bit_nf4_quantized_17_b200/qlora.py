@@ -35,7 +35,8 @@ QLORA_KERNEL_QUANTIZE = 0
 QLORA_KERNEL_FUSED_FWD = 1
 QLORA_KERNEL_FUSED_DGRAD = 2
 QLORA_KERNEL_LORA_GEMM = 3
-QLORA_KERNEL_KINDS = 4
+QLORA_KERNEL_MERGE = 4
+QLORA_KERNEL_KINDS = 5
 
 _DTYPE = {torch.float32: QLORA_F32, torch.bfloat16: QLORA_BF16}
 
@@ -82,6 +83,7 @@ def lib():
             "qlora_linear_bwd": (ctypes.c_int, [pq, vp, vp, i32, f32, vp, vp, vp, i64, vp, vp, vp,
                                                 i32, vp, sz, vp]),
             "qlora_check": (ctypes.c_int, [vp, vp]),
+            "qlora_merge": (ctypes.c_int, [pq, vp, vp, i32, f32, vp, vp]),
             "qlora_launch_count": (ctypes.c_uint64, []),
             "qlora_timing_begin": (ctypes.c_int, [ctypes.c_uint32, i32]),
             "qlora_timing_end": (ctypes.c_int, [ctypes.POINTER(ctypes.c_float),
@@ -245,6 +247,17 @@ def qlora_linear_bwd(q, A, B, alpha, X, U, dY, dX=None, dA=None, dB=None, accumu
 
 def qlora_launch_count():
     return int(lib().qlora_launch_count())
+
+
+def qlora_merge(q, A, B, alpha, out=None, stream=None):
+    """W_merged = bf16(dequant(W) + (alpha / r) B A) as a new (or given) bf16 tensor."""
+    r = A.shape[0]
+    out = out if out is not None else torch.empty((q.rows, q.cols), dtype=torch.bfloat16,
+                                                  device=A.device)
+    st = q.struct
+    _ok(lib().qlora_merge(ctypes.byref(st), _ptr(A), _ptr(B), r, float(alpha), _ptr(out),
+                          _stream(stream)), "qlora_merge")
+    return out
 
 
 def qlora_timing_begin(kinds, max_launches=4096):

@@ -146,8 +146,10 @@ qlora_status qlora_linear_workspace(int64_t M, int64_t N, int64_t K, int32_t r,
                                     size_t* fwd_bytes, size_t* bwd_bytes);
 
 /* Forward pass Y = X W^T + s (X A^T) B^T with W dequantised on the fly (a
- * full-precision W is never written to memory).  Requirements: W->cols % 64
- * == 0 and W->blocksize == 64 (else QLORA_ERR_UNSUPPORTED), 1 <= r <= 256,
+ * full-precision W is never written to memory).  Requirements: W->cols a
+ * multiple of W->blocksize, so that no block straddles two rows (else
+ * QLORA_ERR_UNSUPPORTED; every blocksize, double-quantisation setting and
+ * table of qlora_quantize is accepted), 1 <= r <= 256,
  * M >= 0 (M = 0 is a no-op).  Device buffers: A (r x K bf16), B (N x r bf16),
  * X (M x K bf16), Y (M x N bf16, written), U_save (M x r fp32, written with
  * X A^T; may be NULL), workspace (>= fwd_bytes). */
@@ -166,6 +168,19 @@ qlora_status qlora_linear_bwd(const qlora_nf4* W, const void* A, const void* B,
                               const void* dY, int64_t M, void* dX, float* dA,
                               float* dB, int32_t accumulate, void* workspace,
                               size_t workspace_bytes, void* stream);
+
+/* Merge a trained adapter into a restored 16-bit weight ("LoRA 与 QLoRA：把
+ * 大模型微调拆成可负担的工程", section 3: after training B A has the shape of
+ * W and is added to it; 4-bit storage cannot take the update):
+ *   W_out[n][k] = bf16( fp32(level[idx] * s_hat) + (alpha / r) sum_j B[n][j] A[j][k] )
+ * with the rank-r sum accumulated in fp32 and one final rounding to bf16.
+ * Device buffers: A (r x K bf16), B (N x r bf16), W_out (N x K bf16,
+ * written; 16-byte aligned).  Requirements as for qlora_linear_fwd (W->cols a
+ * multiple of W->blocksize, 1 <= r <= 256); errors QLORA_ERR_NULL, _ALIGN,
+ * _SHAPE, _UNSUPPORTED, _CUDA.  Stream-ordered; allocates nothing.  The
+ * result can be quantised again with qlora_quantize. */
+qlora_status qlora_merge(const qlora_nf4* W, const void* A, const void* B, int32_t r,
+                         float alpha, void* W_out, void* stream);
 
 /* Synchronise `stream`, then return and clear the device status word that
  * calls given this workspace wrote (QLORA_OK if none). */
@@ -193,7 +208,8 @@ typedef enum {
   QLORA_KERNEL_FUSED_FWD = 1,    /* fused dequant GEMM of the forward pass */
   QLORA_KERNEL_FUSED_DGRAD = 2,  /* fused dequant GEMM of dX */
   QLORA_KERNEL_LORA_GEMM = 3,    /* tensor-core rank-r GEMMs (U, V, dA, dB) */
-  QLORA_KERNEL_KINDS = 4
+  QLORA_KERNEL_MERGE = 4,        /* qlora_merge */
+  QLORA_KERNEL_KINDS = 5
 } qlora_kernel_kind;
 qlora_status qlora_timing_begin(uint32_t kind_mask, int32_t max_launches);
 qlora_status qlora_timing_end(float* ms, int32_t* launches);

@@ -16,6 +16,9 @@ What it computes, and where the method is stated:
   backward pass dX, dA, dB with no gradient for W ("LoRA 与 QLoRA：把大模型
   微调拆成可负担的工程", section 2 and section 6; "QLoRA技术从入门到精通",
   section 3(2) and 3(3)).
+  ``merge_weight`` is W_hat + (alpha/r) B A, the update merged into a
+  restored 16-bit weight ("LoRA 与 QLoRA：把大模型微调拆成可负担的工程",
+  section 3).
 * ``bf16.py``  - the bf16 <-> fp32 conversions; the products use the
   dequantised weight rounded to bf16 (``compute_weight``), the compute dtype
   the pages name.
@@ -48,7 +51,7 @@ from .nf4 import (
     compute_weight,
     storage_bits,
 )
-from .linear import lora_scale, linear_fwd, linear_bwd
+from .linear import lora_scale, linear_fwd, linear_bwd, merge_weight
 
 __all__ = [
     "bf16_bits_to_f32", "f32_to_bf16_bits", "round_to_bf16",

@@ -55,3 +55,18 @@ def linear_bwd(w_hat, a, b, alpha, x, dy):
     db = s * (dy.T @ u)
     da = s * (v.T @ x)
     return dx, da, db
+
+
+def merge_weight(w_hat, a, b, alpha):
+    """W_hat + s B A in fp64: the LoRA update added to the restored weight.
+
+    After training, B A has the shape of W and can be added to it
+    ("LoRA 与 QLoRA：把大模型微调拆成可负担的工程" section 3; "LoRA 与 QLoRA：
+    用一块 GPU 微调大模型" section LoRA); the 4-bit storage cannot absorb it,
+    so the sum goes into a restored 16-bit weight.  The merged bf16 weight is
+    this value rounded once to bf16 (``round_to_bf16``), with W_hat the fp32
+    dequantised weight.
+    """
+    w, a, b = _f64(w_hat), _f64(a), _f64(b)
+    s = lora_scale(alpha, a.shape[0])
+    return w + s * (b @ a)

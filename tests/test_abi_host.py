@@ -113,7 +113,8 @@ def test_linear_argument_errors():
     assert _call_fwd(q, r=257) == Q.QLORA_ERR_SHAPE
     assert _call_fwd(q, M=-1) == Q.QLORA_ERR_SHAPE
     assert _call_fwd(_fake_q(256, 200)) == Q.QLORA_ERR_UNSUPPORTED   # d_in % 64 != 0
-    assert _call_fwd(_fake_q(256, 256, bs=128)) == Q.QLORA_ERR_UNSUPPORTED
+    # blocks must not straddle rows: d_in a multiple of the block size
+    assert _call_fwd(_fake_q(256, 384, bs=256)) == Q.QLORA_ERR_UNSUPPORTED
     assert _call_fwd(q, ws_bytes=16) == Q.QLORA_ERR_WORKSPACE
     # M = 0 passes validation and launches nothing
     assert _call_fwd(q, M=0) == Q.QLORA_OK

@@ -1,0 +1,75 @@
+"""GPU parity of qlora_merge: the adapter merged into a restored bf16 weight.
+
+W_merged = bf16(W_hat + (alpha/r) B A) with W_hat the fp32 dequantised
+weight ("LoRA 与 QLoRA：把大模型微调拆成可负担的工程", section 3).  The library
+accumulates the rank-r update in fp32 and rounds once to bf16: every element
+is within one bf16 ulp of the oracle's exact sum rounded to bf16.  With B = 0
+the result is the compute weight bf16(W_hat) bit for bit.  (That the merged
+weight reproduces the layer's forward pass in exact arithmetic is pinned on
+the oracle.)
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bit_nf4_quantized_17_b200 import qlora as Q
+from bit_nf4_quantized_17_b200 import workloads as WL
+from parity import assert_close, f64
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _bf16_bits(t):
+    return t.view(torch.int16).cpu().numpy().view(np.uint16).astype(np.int32)
+
+
+def _ulp_distance(gpu_bits, ref_f32):
+    ref_bits = oracle.f32_to_bf16_bits(np.asarray(ref_f32, np.float32)).astype(np.uint16).astype(np.int32)
+    # bf16 bit patterns of the same sign order like their values
+    return np.abs(gpu_bits - ref_bits)
+
+
+@pytest.mark.parametrize("bs,dq,table", [(64, 256, Q.QLORA_TABLE_NF4), (128, 0, Q.QLORA_TABLE_UNIFORM)])
+def test_merge_matches_oracle(bs, dq, table):
+    shape = WL.WORKLOADS["attn_4096"].linears[0]
+    inp = WL.linear_inputs(shape, 8, 5)
+    W, A, B, X = inp["W"], inp["A"], inp["B"], inp["X"]
+    B = WL.randn(B.shape, 0.05, 9, torch.bfloat16)
+    levels = oracle.uniform_levels() if table == Q.QLORA_TABLE_UNIFORM else oracle.nf4_levels()
+    q = Q.qlora_quantize(W.to(DEV), blocksize=bs, dq_blocksize=dq, table=table)
+    out = Q.qlora_merge(q, A.to(DEV), B.to(DEV), shape.alpha)
+    torch.cuda.synchronize()
+    ref = oracle.quantize(W.float().numpy(), bs, dq, levels=levels)
+    w_hat = oracle.dequantize(ref).reshape(W.shape)
+    exact = oracle.merge_weight(w_hat, A.float().numpy(), B.float().numpy(), shape.alpha)
+    # Bound: one bf16 ulp of the exact value, plus the fp32 error of the sum
+    # (r products, the scaling and the addition, each rounded: (r + 2) 2^-24
+    # of the magnitudes summed), which dominates only where W_hat and the
+    # update nearly cancel.
+    r = A.shape[0]
+    s = oracle.lora_scale(shape.alpha, r)
+    mag = np.abs(w_hat.astype(np.float64)) + s * (np.abs(B.float().numpy()).astype(np.float64)
+                                                  @ np.abs(A.float().numpy()).astype(np.float64))
+    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(exact), 1e-38))) - 7)
+    err = np.abs(f64(out) - exact)
+    assert np.all(err <= ulp + (r + 2) * 2.0 ** -24 * mag)
+    # and nearly always the same bf16 as the exact value rounded once
+    dist = _ulp_distance(_bf16_bits(out), exact.astype(np.float32))
+    assert np.mean(dist == 0) > 0.99
+    # used as a plain bf16 weight, it gives the product of the oracle's merged
+    # weight rounded to bf16 (the merged layer's output, at the bf16 tolerance)
+    merged_bf16 = oracle.round_to_bf16(exact.astype(np.float32)).astype(np.float64)
+    assert_close(f64(X) @ f64(out).T, f64(X) @ merged_bf16.T, "X W_merged^T")
+
+
+def test_merge_with_zero_b_is_the_compute_weight():
+    W = WL.randn((192, 512), 0.02, 11, torch.bfloat16)
+    A = WL.randn((8, 512), 0.35, 12, torch.bfloat16)
+    q = Q.qlora_quantize(W.to(DEV))
+    out = Q.qlora_merge(q, A.to(DEV), torch.zeros((192, 8), dtype=torch.bfloat16, device=DEV), 16.0)
+    torch.cuda.synchronize()
+    ref = oracle.compute_weight(oracle.quantize(W.float().numpy(), 64, 256)).reshape(192, 512)
+    assert np.array_equal(out.float().cpu().numpy(), ref)

@@ -94,3 +94,20 @@ def test_backward_matches_central_finite_differences():
     np.testing.assert_allclose(dx, fd("x_", x), rtol=1e-7, atol=1e-8)
     np.testing.assert_allclose(da, fd("a_", a), rtol=1e-7, atol=1e-8)
     np.testing.assert_allclose(db, fd("b_", b), rtol=1e-7, atol=1e-8)
+
+
+def test_merge_weight_pins():
+    rng = np.random.default_rng(4)
+    w = (rng.standard_normal((24, 64)) * 0.02).astype(np.float32)
+    a, x = _rand(rng, 4, 64), _rand(rng, 5, 64)
+    # B = 0: the merged weight is the restored weight itself
+    assert np.array_equal(oracle.merge_weight(w, a, np.zeros((24, 4), np.float32), 8.0),
+                          w.astype(np.float64))
+    # the merged weight reproduces the forward pass of the unmerged layer
+    b = _rand(rng, 24, 4, scale=0.1)
+    y, _ = oracle.linear_fwd(w, a, b, 8.0, x)
+    merged = oracle.merge_weight(w, a, b, 8.0)
+    assert np.allclose(x.astype(np.float64) @ merged.T, y, rtol=1e-12, atol=1e-12)
+    # the update has rank at most r: removing it from the merged weight gives W back
+    assert np.allclose(merged - w, (merged - w) @ np.linalg.pinv(a.astype(np.float64)) @ a,
+                       atol=1e-12)
