@@ -482,6 +482,86 @@ def run_ours(args):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------- other workloads -------
+
+CONFIGS = {  # --workload name: (workload, linear indices, tokens, input sets, description)
+    "single_256": ("single_256", [0], 16, 3,
+                   "single linear 256x256 fp32 W, r=8 alpha=16, 16 tokens"),
+    "mlp_8192": ("mlp_11008", [0, 1], 8192, 2,
+                 "7B MLP gate/up 4096->11008 and down 11008->4096, r=64 alpha=16, 8192 tokens"),
+    "stack_7b_layer": ("stack_7b", list(range(7)), 2048, 2,
+                       "one layer of the 7B stack (q,k,v,o 4096^2, gate/up 11008x4096, down "
+                       "4096x11008), r=16 alpha=32, 2048 tokens; the stack is 32 such layers"),
+    "stack_65b_layer": ("stack_65b", list(range(7)), 2048, 2,
+                        "one layer of the 65B-shaped stack (8192^2 x4, 22016x8192 x2, "
+                        "8192x22016), r=64 alpha=16, 2048 tokens; the stack is 80 such layers"),
+}
+
+
+def run_config(args):
+    """One step over the linears of a workload: quantise all, forward in
+    order, backward in reverse order (layer-by-layer chaining)."""
+    from bit_nf4_quantized_17_b200 import dp
+    from bit_nf4_quantized_17_b200 import qlora as Q
+    from bit_nf4_quantized_17_b200 import workloads as WL
+
+    name, idx, M, n_sets, desc = CONFIGS[args.workload]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks = measured_peaks()
+    shapes = [WL.WORKLOADS[name].linears[j] for j in idx]
+    sets = [[InputSet(sh, M, WL.stack_seed(0, j) + 1000 * i, 0, dev, Q, WL, dp)
+             for sh, j in zip(shapes, idx)] for i in range(n_sets)]
+    flops = sum(fwd_bwd_flops(M, sh.d_out, sh.d_in, sh.r) for sh in shapes)
+    fused_f = sum(fwd_flops(M, sh.d_out, sh.d_in, sh.r) for sh in shapes)
+    fused_b = sum(2 * M * sh.d_out * sh.d_in + 2 * M * sh.d_in * sh.r for sh in shapes)
+
+    def step(group):
+        for s, sh in zip(group, shapes):
+            Q.qlora_quantize(s.W, out=s.q, workspace=s.qws, check=False)
+        for s, sh in zip(group, shapes):
+            Q.qlora_linear_fwd(s.q, s.A, s.B, sh.alpha, s.X, Y=s.Y, U_save=s.U, workspace=s.fws)
+        for s, sh in reversed(list(zip(group, shapes))):
+            Q.qlora_linear_bwd(s.q, s.A, s.B, sh.alpha, s.X, s.U, s.dY, dX=s.dX, dA=s.dA,
+                               dB=s.dB, workspace=s.bws)
+
+    for i in range(args.warmup):
+        step(sets[i % n_sets])
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(0) as clk:
+        torch.cuda.synchronize()
+        Q.qlora_timing_begin((Q.QLORA_KERNEL_FUSED_FWD, Q.QLORA_KERNEL_FUSED_DGRAD),
+                             max_launches=4 * len(shapes) * args.steps)
+        start.record()
+        for i in range(args.steps):
+            step(sets[i % n_sets])
+        end.record()
+        torch.cuda.synchronize()
+        kt = Q.qlora_timing_end()
+    ms = start.elapsed_time(end) / args.steps
+    value = flops / (ms * 1e-3) / 1e12
+    t_f = kt[Q.QLORA_KERNEL_FUSED_FWD][0] / args.steps * 1e-3
+    t_b = kt[Q.QLORA_KERNEL_FUSED_DGRAD][0] / args.steps * 1e-3
+    nf4 = sum(nf4_bytes(sh.d_out, sh.d_in) for sh in shapes)
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,.) tensors of the workload's shapes)",
+        "config": {"workload": f"{args.workload}: {desc}; step = quantise + fwd + bwd of "
+                               "every linear", "global_batch": M,
+                   "l2": f"{n_sets} rotating input sets"},
+        "frac_of_bf16_peak": round(value / peaks["bf16_sustained"], 4),
+        "fused_fwd_tflops": round(fused_f / t_f / 1e12, 2) if t_f > 0 else None,
+        "fused_dgrad_tflops": round(fused_b / t_b / 1e12, 2) if t_b > 0 else None,
+        "fused_share": round((t_f + t_b) / (ms * 1e-3), 4),
+        "nf4_weight_gbs": round(2 * nf4 / (ms * 1e-3) / 1e9, 1),
+        "clocks": clk.summary(), "peaks": peaks,
+    }
+    print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------ reference arm ----
 
 def run_reference(args):
@@ -540,11 +620,15 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--workload", default=WORKLOAD, choices=[WORKLOAD] + sorted(CONFIGS),
+                    help="another workload of the problem (one GPU, our arm only)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload != WORKLOAD:
+        run_config(args)
     else:
         run_ours(args)
 

@@ -178,6 +178,51 @@ qlora_status qlora_dequantize(const qlora_nf4* q, void* W_out, int32_t out_dtype
   return launch_dequantize(*q, *t, W_out, out_dtype, static_cast<cudaStream_t>(stream));
 }
 
+qlora_status qlora_adamw(float* param, void* param_bf16, const float* grad, float* m, float* v,
+                         int64_t n, int32_t step, float lr, float beta1, float beta2, float eps,
+                         float weight_decay, float grad_scale, void* stream) {
+  if (n < 0 || step < 1) return QLORA_ERR_SHAPE;
+  if (n == 0) return QLORA_OK;
+  if (!param || !grad || !m || !v) return QLORA_ERR_NULL;
+  if (!aligned16(param) || !aligned16(grad) || !aligned16(m) || !aligned16(v) ||
+      !aligned16(param_bf16))
+    return QLORA_ERR_ALIGN;  // (a NULL param_bf16 counts as aligned)
+  if (!(beta1 >= 0.0f && beta1 < 1.0f) || !(beta2 >= 0.0f && beta2 < 1.0f) || !(eps > 0.0f) ||
+      !(lr >= 0.0f))
+    return QLORA_ERR_UNSUPPORTED;
+  return launch_adamw(param, param_bf16, grad, m, v, n, step, lr, beta1, beta2, eps, weight_decay,
+                      grad_scale, static_cast<cudaStream_t>(stream));
+}
+
+qlora_status qlora_paged_alloc(size_t bytes, void** ptr) {
+  if (!ptr) return QLORA_ERR_NULL;
+  *ptr = nullptr;
+  if (bytes == 0) return QLORA_ERR_SHAPE;
+  void* p = nullptr;
+  if (cudaMallocManaged(&p, bytes, cudaMemAttachGlobal) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (cudaMemset(p, 0, bytes) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+    cudaFree(p);
+    return QLORA_ERR_CUDA;
+  }
+  *ptr = p;
+  return QLORA_OK;
+}
+
+qlora_status qlora_paged_prefetch(void* ptr, size_t bytes, int32_t to_device, void* stream) {
+  if (!ptr) return QLORA_ERR_NULL;
+  if (bytes == 0) return QLORA_ERR_SHAPE;
+  int dev = cudaCpuDeviceId;
+  if (to_device && cudaGetDevice(&dev) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (cudaMemPrefetchAsync(ptr, bytes, dev, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  return QLORA_OK;
+}
+
+qlora_status qlora_paged_free(void* ptr) {
+  if (!ptr) return QLORA_OK;
+  return cudaFree(ptr) == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
 qlora_status qlora_merge(const qlora_nf4* W, const void* A, const void* B, int32_t r,
                          float alpha, void* W_out, void* stream) {
   if (!W || !A || !B || !W_out) return QLORA_ERR_NULL;

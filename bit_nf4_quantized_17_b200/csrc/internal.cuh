@@ -60,6 +60,11 @@ qlora_status launch_quantize(const void* W, int32_t w_dtype, const qlora_nf4& q,
 qlora_status launch_dequantize(const qlora_nf4& q, const LevelTable& t, void* out,
                                int32_t out_dtype, cudaStream_t s);
 
+// adamw.cu: one AdamW step over n fp32 parameters (and their bf16 copy)
+qlora_status launch_adamw(float* p, void* p16, const float* g, float* m, float* v, int64_t n,
+                          int32_t step, float lr, float beta1, float beta2, float eps,
+                          float weight_decay, float grad_scale, cudaStream_t s);
+
 // merge.cu: W_out = bf16(dequant(W) + (alpha / r) B A)
 qlora_status launch_merge(const qlora_nf4& q, const LevelTable& t, const void* A, const void* B,
                           int32_t r, float alpha, void* out, cudaStream_t s);

@@ -40,6 +40,7 @@ class GradBucket:
     def __init__(self, r, d_in, d_out, device):
         na = r * d_in
         off_b = -(-na // _ALIGN) * _ALIGN
+        self.off_b = off_b
         self.flat = torch.zeros(off_b + d_out * r, dtype=torch.float32, device=device)
         self.dA = self.flat[:na].view(r, d_in)
         self.dB = self.flat[off_b:off_b + d_out * r].view(d_out, r)

@@ -84,6 +84,11 @@ def lib():
                                                 i32, vp, sz, vp]),
             "qlora_check": (ctypes.c_int, [vp, vp]),
             "qlora_merge": (ctypes.c_int, [pq, vp, vp, i32, f32, vp, vp]),
+            "qlora_paged_alloc": (ctypes.c_int, [ctypes.c_size_t, ctypes.POINTER(ctypes.c_void_p)]),
+            "qlora_paged_prefetch": (ctypes.c_int, [vp, ctypes.c_size_t, i32, vp]),
+            "qlora_paged_free": (ctypes.c_int, [vp]),
+            "qlora_adamw": (ctypes.c_int, [vp, vp, vp, vp, vp, i64, i32, f32, f32, f32, f32, f32,
+                                           f32, vp]),
             "qlora_launch_count": (ctypes.c_uint64, []),
             "qlora_timing_begin": (ctypes.c_int, [ctypes.c_uint32, i32]),
             "qlora_timing_end": (ctypes.c_int, [ctypes.POINTER(ctypes.c_float),
@@ -258,6 +263,52 @@ def qlora_merge(q, A, B, alpha, out=None, stream=None):
     _ok(lib().qlora_merge(ctypes.byref(st), _ptr(A), _ptr(B), r, float(alpha), _ptr(out),
                           _stream(stream)), "qlora_merge")
     return out
+
+
+def qlora_adamw(param, grad, m, v, step, lr, beta1=0.9, beta2=0.999, eps=1e-8,
+                weight_decay=0.0, grad_scale=1.0, param_bf16=None, stream=None):
+    """One AdamW step in place over flat fp32 tensors (param, m, v updated);
+    param_bf16, if given, receives bf16(param)."""
+    n = param.numel()
+    for t in (param, grad, m, v):
+        assert t.dtype == torch.float32 and t.is_contiguous() and t.numel() == n
+    _ok(lib().qlora_adamw(_ptr(param), _ptr(param_bf16), _ptr(grad), _ptr(m), _ptr(v), n,
+                          int(step), float(lr), float(beta1), float(beta2), float(eps),
+                          float(weight_decay), float(grad_scale), _stream(stream)), "qlora_adamw")
+
+
+class _PagedBlock:
+    """Owner of one qlora_paged_alloc block, exposed to torch through the CUDA
+    array interface; the block is freed when the last tensor on it goes."""
+
+    def __init__(self, numel, dtype):
+        self.nbytes = int(numel) * torch.empty((), dtype=dtype).element_size()
+        ptr = ctypes.c_void_p()
+        _ok(lib().qlora_paged_alloc(self.nbytes, ctypes.byref(ptr)), "qlora_paged_alloc")
+        self.ptr = ptr.value
+        typestr = {torch.float32: "<f4", torch.uint8: "|u1"}[dtype]
+        self.__cuda_array_interface__ = {
+            "shape": (int(numel),), "typestr": typestr, "data": (self.ptr, False),
+            "version": 3, "strides": None, "stream": None}
+
+    def __del__(self):
+        if getattr(self, "ptr", None) and _lib is not None:
+            _lib.qlora_paged_free(ctypes.c_void_p(self.ptr))
+            self.ptr = None
+
+
+def qlora_paged_empty(numel, dtype=torch.float32):
+    """A zero-filled 1-D tensor of `numel` elements in managed (paged) memory
+    from qlora_paged_alloc; it keeps its block alive."""
+    if dtype not in (torch.float32, torch.uint8):
+        raise ValueError("paged tensors are fp32 or uint8")
+    return torch.as_tensor(_PagedBlock(numel, dtype), device="cuda")
+
+
+def qlora_paged_prefetch(t, to_device=True, stream=None):
+    """Enqueue a migration of tensor `t`'s pages to the current GPU or to host memory."""
+    _ok(lib().qlora_paged_prefetch(_ptr(t), t.numel() * t.element_size(), 1 if to_device else 0,
+                                   _stream(stream)), "qlora_paged_prefetch")
 
 
 def qlora_timing_begin(kinds, max_launches=4096):

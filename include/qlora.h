@@ -24,7 +24,8 @@
  *   - Pointers named "device" are CUDA device pointers, 16-byte aligned.  The
  *     caller owns and allocates every buffer (sizes from the *_sizes and
  *     *_workspace queries); the library never allocates, frees or keeps a
- *     pointer after a call returns.
+ *     pointer after a call returns - except qlora_paged_alloc and
+ *     qlora_paged_free, whose whole job is that.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
  *     stream-ordered and asynchronous: they return after enqueueing work.
  *   - Argument errors are found on the host and returned before any launch.
@@ -181,6 +182,40 @@ qlora_status qlora_linear_bwd(const qlora_nf4* W, const void* A, const void* B,
  * result can be quantised again with qlora_quantize. */
 qlora_status qlora_merge(const qlora_nf4* W, const void* A, const void* B, int32_t r,
                          float alpha, void* W_out, void* stream);
+
+/* One AdamW step (Adam with decoupled weight decay) over n adapter
+ * parameters - the optimiser that updates only A and B ("QLoRA技术从入门到精
+ * 通", section 3(3)).  For step >= 1, per element, g' = grad_scale * grad:
+ *   m = beta1 m + (1 - beta1) g',  v = beta2 v + (1 - beta2) g'^2,
+ *   param -= lr (m / (1 - beta1^step) / (sqrt(v / (1 - beta2^step)) + eps)
+ *                + weight_decay param),
+ * then param_bf16 = bf16(param) when param_bf16 is not NULL.  Device buffers
+ * (any device-accessible memory, managed memory included): param, grad, m, v
+ * (n fp32 each; param, m, v updated in place), param_bf16 (n bf16, written).
+ * All 16-byte aligned.  The flat dA/dB buffer of a data-parallel step can be
+ * passed whole.  Errors: QLORA_ERR_NULL, _ALIGN, _SHAPE (n < 0, step < 1),
+ * _UNSUPPORTED (beta outside [0, 1), eps <= 0, lr < 0), _CUDA. */
+qlora_status qlora_adamw(float* param, void* param_bf16, const float* grad, float* m, float* v,
+                         int64_t n, int32_t step, float lr, float beta1, float beta2, float eps,
+                         float weight_decay, float grad_scale, void* stream);
+
+/* Paged optimiser states.  The optimiser moments can live in CUDA managed
+ * (unified) memory, which the driver migrates between host and device pages
+ * on demand, so that they need not stay in HBM ("LoRA 与 QLoRA：把大模型微调
+ * 拆成可负担的工程", section 6.3; "QLoRA 量化微调", paged optimisers).
+ *   qlora_paged_alloc:    `bytes` of managed memory (global attachment,
+ *                         256-byte aligned, zero-filled) into *ptr.
+ *   qlora_paged_prefetch: enqueue on `stream` a migration of [ptr, ptr+bytes)
+ *                         to the current device (to_device != 0) or to host
+ *                         memory (to_device == 0).  Optional: pages that are
+ *                         not resident move on first touch anyway.
+ *   qlora_paged_free:     release a pointer from qlora_paged_alloc (waits for
+ *                         the device, as cudaFree does).  NULL is a no-op.
+ * Errors: QLORA_ERR_NULL, QLORA_ERR_SHAPE (bytes == 0), QLORA_ERR_CUDA
+ * (allocation failed or the device cannot prefetch managed memory). */
+qlora_status qlora_paged_alloc(size_t bytes, void** ptr);
+qlora_status qlora_paged_prefetch(void* ptr, size_t bytes, int32_t to_device, void* stream);
+qlora_status qlora_paged_free(void* ptr);
 
 /* Synchronise `stream`, then return and clear the device status word that
  * calls given this workspace wrote (QLORA_OK if none). */

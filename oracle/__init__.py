@@ -19,6 +19,8 @@ What it computes, and where the method is stated:
   ``merge_weight`` is W_hat + (alpha/r) B A, the update merged into a
   restored 16-bit weight ("LoRA 与 QLoRA：把大模型微调拆成可负担的工程",
   section 3).
+* ``optim.py`` - the AdamW step for the adapters (the optimiser that updates
+  only A and B, "QLoRA技术从入门到精通", section 3(3)).
 * ``bf16.py``  - the bf16 <-> fp32 conversions; the products use the
   dequantised weight rounded to bf16 (``compute_weight``), the compute dtype
   the pages name.
@@ -52,11 +54,12 @@ from .nf4 import (
     storage_bits,
 )
 from .linear import lora_scale, linear_fwd, linear_bwd, merge_weight
+from .optim import adamw_step
 
 __all__ = [
     "bf16_bits_to_f32", "f32_to_bf16_bits", "round_to_bf16",
     "nf4_levels", "nf4_raw_quantiles", "uniform_levels", "nearest_level",
     "block_absmax", "pack_nibbles", "unpack_nibbles", "fixed_point_mean",
     "double_quantize", "dequantize_scales", "block_scales", "quantize", "dequantize", "compute_weight",
-    "storage_bits", "lora_scale", "linear_fwd", "linear_bwd",
+    "storage_bits", "lora_scale", "linear_fwd", "linear_bwd", "merge_weight", "adamw_step",
 ]

@@ -147,3 +147,29 @@ def test_timing_hook_rejects_bad_requests_without_cuda():
     assert L.qlora_timing_begin(0x3, 65537) == Q.QLORA_ERR_SHAPE
     # ending while timing is off
     assert L.qlora_timing_end(None, None) == Q.QLORA_ERR_UNSUPPORTED
+
+
+def test_adamw_and_paged_argument_errors_without_cuda():
+    L = Q.lib()
+    P = ctypes.c_void_p
+    a, b = P(0x20000), P(0x30000)
+
+    def adamw(p=a, p16=None, g=b, m=a, v=b, n=8, step=1, lr=1e-3, b1=0.9, b2=0.999, eps=1e-8):
+        return L.qlora_adamw(p, p16, g, m, v, n, step, lr, b1, b2, eps, 0.0, 1.0, None)
+
+    assert adamw(n=0) == Q.QLORA_OK          # nothing to do: returns before any launch
+    assert adamw(n=-1) == Q.QLORA_ERR_SHAPE
+    assert adamw(step=0) == Q.QLORA_ERR_SHAPE
+    assert adamw(g=None) == Q.QLORA_ERR_NULL
+    assert adamw(m=P(0x20004)) == Q.QLORA_ERR_ALIGN
+    assert adamw(p16=P(0x40002)) == Q.QLORA_ERR_ALIGN
+    assert adamw(b2=1.0) == Q.QLORA_ERR_UNSUPPORTED
+    assert adamw(b1=-0.1) == Q.QLORA_ERR_UNSUPPORTED
+    assert adamw(eps=0.0) == Q.QLORA_ERR_UNSUPPORTED
+    assert adamw(lr=float("nan")) == Q.QLORA_ERR_UNSUPPORTED
+    out = P(1)
+    assert L.qlora_paged_alloc(0, ctypes.byref(out)) == Q.QLORA_ERR_SHAPE and out.value is None
+    assert L.qlora_paged_alloc(64, None) == Q.QLORA_ERR_NULL
+    assert L.qlora_paged_prefetch(None, 64, 1, None) == Q.QLORA_ERR_NULL
+    assert L.qlora_paged_prefetch(a, 0, 1, None) == Q.QLORA_ERR_SHAPE
+    assert L.qlora_paged_free(None) == Q.QLORA_OK
