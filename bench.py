@@ -270,6 +270,39 @@ def time_decode(Q, WL, dev, peaks, steps=30, warmup=5):
         kt = Q.qlora_timing_end()
         t_f = statistics.median(e[0].elapsed_time(e[1]) for e in evs) * 1e-3
         t_b = statistics.median(e[1].elapsed_time(e[2]) for e in evs) * 1e-3
+        # the same calls replayed from CUDA graphs (one forward and one
+        # backward graph per weight copy), as a decode loop would run them:
+        # the host's per-call cost leaves the measurement
+        graphs = []
+        cap = torch.cuda.Stream()
+        cap.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(cap):
+            for c in range(8):
+                gf, gb = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+                with torch.cuda.graph(gf, stream=cap):
+                    Q.qlora_linear_fwd(copies[c], A, B, shape.alpha, X, Y=Y, U_save=U, workspace=fws)
+                with torch.cuda.graph(gb, stream=cap):
+                    Q.qlora_linear_bwd(copies[c], A, B, shape.alpha, X, U, dY, dX=dX, dA=dA, dB=dB,
+                                       workspace=bws)
+                graphs.append((gf, gb))
+        torch.cuda.current_stream().wait_stream(cap)
+        torch.cuda.synchronize()
+        gevs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        for i in range(warmup + steps):
+            gf, gb = graphs[i % 8]
+            e = gevs[i - warmup] if i >= warmup else None
+            if e:
+                e[0].record()
+            gf.replay()
+            if e:
+                e[1].record()
+            gb.replay()
+            if e:
+                e[2].record()
+        torch.cuda.synchronize()
+        g_f = statistics.median(e[0].elapsed_time(e[1]) for e in gevs) * 1e-3
+        g_b = statistics.median(e[1].elapsed_time(e[2]) for e in gevs) * 1e-3
+        del graphs
         wb = nf4_bytes(N, K)
         # the fused kernels alone: NF4 bytes + activations in/out + adapter
         # (algorithmic HBM bytes of one launch) / average launch time
@@ -287,6 +320,9 @@ def time_decode(Q, WL, dev, peaks, steps=30, warmup=5):
             "fwd_nf4_gbs": round(wb / t_f / 1e9, 1), "bwd_nf4_gbs": round(wb / t_b / 1e9, 1),
             "fwd_frac_hbm": round(wb / t_f / 1e9 / peaks["hbm"], 4),
             "bwd_frac_hbm": round(wb / t_b / 1e9 / peaks["hbm"], 4),
+            "graph_fwd_us": round(g_f * 1e6, 2), "graph_bwd_us": round(g_b * 1e6, 2),
+            "graph_fwd_frac_hbm": round(wb / g_f / 1e9 / peaks["hbm"], 4),
+            "graph_bwd_frac_hbm": round(wb / g_b / 1e9 / peaks["hbm"], 4),
             "kernels": fused,
         }
     out["workload"] = "mlp gate/up 11008x4096, r=64, alpha=16; NF4 bytes per pass " \

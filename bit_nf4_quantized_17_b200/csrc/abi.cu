@@ -273,7 +273,7 @@ qlora_status qlora_linear_fwd(const qlora_nf4* W, const void* A, const void* B, 
   if (!Y) return QLORA_ERR_NULL;
   if (!aligned16(Y) || (U_save && !aligned16(U_save))) return QLORA_ERR_ALIGN;
   return linear_forward(*W, *level_table(W->table), A, B, r, alpha, X, M, Y, U_save, workspace,
-                        static_cast<cudaStream_t>(stream));
+                        static_cast<cudaStream_t>(stream), LoraOpts{r, nullptr, nullptr, nullptr, 1.0f});
 }
 
 qlora_status qlora_linear_bwd(const qlora_nf4* W, const void* A, const void* B, int32_t r,
@@ -296,7 +296,113 @@ qlora_status qlora_linear_bwd(const qlora_nf4* W, const void* A, const void* B, 
     return QLORA_OK;
   }
   return linear_backward(*W, *level_table(W->table), A, B, r, alpha, X, U, dY, M, dX, dA, dB,
-                         accumulate != 0, workspace, s);
+                         accumulate != 0, workspace, s, LoraOpts{r, nullptr, nullptr, nullptr, 1.0f});
+}
+
+static qlora_status check_multi(const qlora_nf4* W, int32_t n_adapters, int32_t r,
+                                const int32_t* adapter, int64_t M) {
+  if (n_adapters < 1 || r < 1 || static_cast<int64_t>(n_adapters) * r > 256) return QLORA_ERR_SHAPE;
+  if (M > 0 && !adapter) return QLORA_ERR_NULL;
+  if (reinterpret_cast<uintptr_t>(adapter) % 4 != 0) return QLORA_ERR_ALIGN;
+  if (!linear_multi_supported(M, W->rows, W->cols, n_adapters * r)) return QLORA_ERR_UNSUPPORTED;
+  return QLORA_OK;
+}
+
+static qlora_status opts_of(const qlora_adapter_opts* x, const qlora_nf4* W, int32_t r, int64_t M,
+                            LoraOpts* o, int32_t* rt) {
+  const int32_t n = x ? x->n_adapters : 1;
+  if (n < 1 || r < 1 || static_cast<int64_t>(n) * r > 256) return QLORA_ERR_SHAPE;
+  *rt = n * r;
+  *o = LoraOpts{r, nullptr, nullptr, nullptr, 1.0f};
+  if (!x) return QLORA_OK;
+  if (x->adapter || n > 1) {
+    qlora_status st = check_multi(W, n, r, x->adapter, M);
+    if (st != QLORA_OK) return st;
+    o->seg = x->adapter;
+  }
+  if (x->keep_mask) {
+    if (!(x->dropout_p >= 0.0f && x->dropout_p < 1.0f)) return QLORA_ERR_UNSUPPORTED;
+    if (M > 0 && !x->x_drop) return QLORA_ERR_NULL;
+    if (!aligned16(x->x_drop)) return QLORA_ERR_ALIGN;
+    if (!linear_multi_supported(M, W->rows, W->cols, *rt)) return QLORA_ERR_UNSUPPORTED;
+    o->mask = x->keep_mask;
+    o->x_drop = x->x_drop;
+    o->keep = 1.0f / (1.0f - x->dropout_p);
+  }
+  return QLORA_OK;
+}
+
+qlora_status qlora_linear_fwd_ex(const qlora_nf4* W, const void* A, const void* B, int32_t r,
+                                 float alpha, const qlora_adapter_opts* opts, const void* X,
+                                 int64_t M, void* Y, float* U_save, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  if (!W) return QLORA_ERR_NULL;
+  LoraOpts o{};
+  int32_t rt = 0;
+  qlora_status st = opts_of(opts, W, r, M, &o, &rt);
+  if (st != QLORA_OK) return st;
+  if ((st = check_linear(W, A, B, rt, M, X, workspace, workspace_bytes, false)) != QLORA_OK)
+    return st;
+  if (M == 0) return QLORA_OK;
+  if (!Y) return QLORA_ERR_NULL;
+  if (!aligned16(Y) || (U_save && !aligned16(U_save))) return QLORA_ERR_ALIGN;
+  return linear_forward(*W, *level_table(W->table), A, B, rt, alpha, X, M, Y, U_save, workspace,
+                        static_cast<cudaStream_t>(stream), o);
+}
+
+qlora_status qlora_linear_bwd_ex(const qlora_nf4* W, const void* A, const void* B, int32_t r,
+                                 float alpha, const qlora_adapter_opts* opts, const void* X,
+                                 const float* U, const void* dY, int64_t M, void* dX, float* dA,
+                                 float* dB, int32_t accumulate, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  if (!W) return QLORA_ERR_NULL;
+  LoraOpts o{};
+  int32_t rt = 0;
+  qlora_status st = opts_of(opts, W, r, M, &o, &rt);
+  if (st != QLORA_OK) return st;
+  if ((st = check_linear(W, A, B, rt, M, X, workspace, workspace_bytes, true)) != QLORA_OK)
+    return st;
+  if ((M > 0 && !dY) || !dA || !dB) return QLORA_ERR_NULL;
+  if (!aligned16(dY) || !aligned16(dA) || !aligned16(dB) || (dX && !aligned16(dX)) ||
+      (U && !aligned16(U)))
+    return QLORA_ERR_ALIGN;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (M == 0) {
+    if (accumulate) return QLORA_OK;
+    if (cudaMemsetAsync(dA, 0, sizeof(float) * rt * W->cols, s) != cudaSuccess ||
+        cudaMemsetAsync(dB, 0, sizeof(float) * rt * W->rows, s) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+    return QLORA_OK;
+  }
+  return linear_backward(*W, *level_table(W->table), A, B, rt, alpha, X, U, dY, M, dX, dA, dB,
+                         accumulate != 0, workspace, s, o);
+}
+
+qlora_status qlora_linear_fwd_multi(const qlora_nf4* W, const void* A, const void* B,
+                                    int32_t n_adapters, int32_t r, float alpha,
+                                    const int32_t* adapter, const void* X, int64_t M, void* Y,
+                                    float* U_save, void* workspace, size_t workspace_bytes,
+                                    void* stream) {
+  qlora_adapter_opts x{};
+  x.n_adapters = n_adapters;
+  x.adapter = adapter;
+  if (M > 0 && !adapter) return QLORA_ERR_NULL;
+  return qlora_linear_fwd_ex(W, A, B, r, alpha, &x, X, M, Y, U_save, workspace, workspace_bytes,
+                             stream);
+}
+
+qlora_status qlora_linear_bwd_multi(const qlora_nf4* W, const void* A, const void* B,
+                                    int32_t n_adapters, int32_t r, float alpha,
+                                    const int32_t* adapter, const void* X, const float* U,
+                                    const void* dY, int64_t M, void* dX, float* dA, float* dB,
+                                    int32_t accumulate, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+  qlora_adapter_opts x{};
+  x.n_adapters = n_adapters;
+  x.adapter = adapter;
+  if (M > 0 && !adapter) return QLORA_ERR_NULL;
+  return qlora_linear_bwd_ex(W, A, B, r, alpha, &x, X, U, dY, M, dX, dA, dB, accumulate,
+                             workspace, workspace_bytes, stream);
 }
 
 qlora_status qlora_check(void* workspace, void* stream) {

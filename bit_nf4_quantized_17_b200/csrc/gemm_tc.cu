@@ -441,7 +441,8 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ part, int splits,
                                      int cols, int pcols, int lo, float* o1, int64_t ld1,
                                      int trans1, float a1, int acc1, __nv_bfloat16* o2, int64_t ld2,
                                      float a2, int o2_lo, __nv_bfloat16* o3, int64_t ld3, float a3,
-                                     int o3_lo, int o2_pad) {
+                                     int o3_lo, int o2_pad, const int32_t* __restrict__ seg,
+                                     int seg_cols) {
   const int64_t total = rows * cols;
   const int pad = (o2 && o2_pad) ? o2_lo - cols : 0;
   const int64_t total_pad = rows * 2 * pad;
@@ -475,6 +476,7 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ part, int splits,
         }
       }
     }
+    if (seg && __ldg(seg + i) != j / seg_cols) v = 0.0f;
     reduce_store(v, i, j, o1, ld1, trans1, a1, acc1, o2, ld2, a2, o2_lo, o3, ld3, a3, o3_lo);
   }
 }
@@ -486,7 +488,8 @@ __global__ void splitk_reduce_warp_kernel(const float* __restrict__ part, int sp
                                           int cols, int pcols, int lo, float* o1, int64_t ld1,
                                           int trans1, float a1, int acc1, __nv_bfloat16* o2,
                                           int64_t ld2, float a2, int o2_lo, __nv_bfloat16* o3,
-                                          int64_t ld3, float a3, int o3_lo, int o2_pad) {
+                                          int64_t ld3, float a3, int o3_lo, int o2_pad,
+                                          const int32_t* __restrict__ seg, int seg_cols) {
   const int64_t total = rows * cols;
   const int64_t split_stride = rows * pcols;
   const int lane = threadIdx.x & 31;
@@ -512,6 +515,7 @@ __global__ void splitk_reduce_warp_kernel(const float* __restrict__ part, int sp
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    if (seg && __ldg(seg + i) != j / seg_cols) v = 0.0f;
     if (lane == 0)
       reduce_store(v, i, j, o1, ld1, trans1, a1, acc1, o2, ld2, a2, o2_lo, o3, ld3, a3, o3_lo);
   }
@@ -778,7 +782,8 @@ qlora_status splitk_reduce(const ReduceArgs& a, cudaStream_t s) {
     splitk_reduce_warp_kernel<<<grid, 256, 0, s>>>(
         a.part, a.splits, a.rows, a.cols, a.pcols, a.lo, a.o1, a.ld1, a.trans1 ? 1 : 0, a.a1,
         a.acc1 ? 1 : 0, static_cast<__nv_bfloat16*>(a.o2), a.ld2, a.a2, a.o2_lo,
-        static_cast<__nv_bfloat16*>(a.o3), a.ld3, a.a3, a.o3_lo, a.o2_pad);
+        static_cast<__nv_bfloat16*>(a.o3), a.ld3, a.a3, a.o3_lo, a.o2_pad, a.seg,
+        a.seg ? a.seg_cols : 1);
   } else {
     const int64_t pad_items = (a.o2 && a.o2_pad) ? a.rows * 2 * (a.o2_lo - a.cols) : 0;
     const int grid =
@@ -786,7 +791,8 @@ qlora_status splitk_reduce(const ReduceArgs& a, cudaStream_t s) {
     splitk_reduce_kernel<<<grid, 256, 0, s>>>(
         a.part, a.splits, a.rows, a.cols, a.pcols, a.lo, a.o1, a.ld1, a.trans1 ? 1 : 0, a.a1,
         a.acc1 ? 1 : 0, static_cast<__nv_bfloat16*>(a.o2), a.ld2, a.a2, a.o2_lo,
-        static_cast<__nv_bfloat16*>(a.o3), a.ld3, a.a3, a.o3_lo, a.o2_pad);
+        static_cast<__nv_bfloat16*>(a.o3), a.ld3, a.a3, a.o3_lo, a.o2_pad, a.seg,
+        a.seg ? a.seg_cols : 1);
   }
   return after_launch("splitk_reduce", s);
 }

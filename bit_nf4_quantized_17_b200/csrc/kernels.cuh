@@ -109,10 +109,21 @@ struct ReduceArgs {
   float a3;
   int o3_lo;
   int o2_pad;  // > 0: also write zeros to o2 columns [cols, o2_lo) and [o2_lo + cols, 2 o2_lo)
+  // adapter mask: when set, output (i, j) is kept only if seg[i] == j / seg_cols
+  // (row i = a token, its columns [a seg_cols, (a + 1) seg_cols) = adapter a)
+  const int32_t* seg;
+  int seg_cols;
 };
 qlora_status splitk_reduce(const ReduceArgs& a, cudaStream_t s);
 qlora_status transpose_to_bf16(const void* in, bool in_f32, int64_t rows, int cols, int64_t ld_in,
                                void* out, int64_t ld_out, int lo_rows, cudaStream_t s);
+
+// dropout.cu: X_drop = X (.) D (mask bit (k % 8) of byte m K / 8 + k / 8 keeps
+// X[m][k]; K a multiple of 8), and dX[m][k] += D[m][k] scale (V A)[m][k] in place.
+qlora_status dropout_apply(const void* X, const uint8_t* mask, int64_t M, int64_t K, void* X_drop,
+                           cudaStream_t s);
+qlora_status dropout_dx(void* dX, const float* V, int64_t ldv, const void* A, const uint8_t* mask,
+                        int64_t M, int64_t K, int32_t r, float scale, cudaStream_t s);
 
 // lora_small.cu: LoRA-side kernels for M <= 16 tokens (CUDA cores).
 constexpr int kSmallM = 16;

@@ -55,9 +55,9 @@ TcSplits tc_splits(int64_t M, int64_t N, int64_t K) {
 // Workspace regions of the tensor-core path (byte offsets; the status word is first).
 //   forward   sU [hi | lo] (M x 2*span bf16) | split-K partials
 //   backward  U^T [hi ; lo] (2*r16 x M8 bf16) | B^T (r x N bf16) | sV [hi | lo] |
-//             V^T [hi ; lo] | split-K partials
+//             V^T [hi ; lo] | V (M x r fp32) | split-K partials
 struct TcLayout {
-  size_t su, part_f, fused_f, ut, bt, sv, vt, part_b, fused_b, fwd_end, bwd_end;
+  size_t su, part_f, fused_f, ut, bt, sv, vt, v32, part_b, fused_b, fwd_end, bwd_end;
 };
 
 TcLayout tc_layout(int64_t M, int64_t N, int64_t K, int32_t r) {
@@ -73,7 +73,8 @@ TcLayout tc_layout(int64_t M, int64_t N, int64_t K, int32_t r) {
   L.bt = L.ut + align256(2 * 2 * r16 * mp);
   L.sv = L.bt + align256(2 * r * N);
   L.vt = L.sv + align256(2 * M * 2 * span);
-  L.part_b = L.vt + align256(2 * 2 * r16 * mp);
+  L.v32 = L.vt + align256(2 * 2 * r16 * mp);  // V in fp32, for the dropout-masked dX term
+  L.part_b = L.v32 + align256(sizeof(float) * M * r);
   const int64_t part = std::max(std::max(sp.u * M * r16, sp.v * M * r16),
                                 std::max(sp.db * N * 2 * r16, sp.da * K * 2 * r16));
   L.fused_b = L.part_b + align256(sizeof(float) * part);
@@ -177,27 +178,43 @@ LinearPlan plan_linear(int64_t M, int64_t N, int64_t K, int32_t r) {
     if (_st != QLORA_OK) return _st;      \
   } while (0)
 
+bool linear_multi_supported(int64_t M, int64_t N, int64_t K, int32_t r) {
+  return use_tc(M > 0 ? M : 1, N, K, r);  // (M = 0 is a no-op on every path)
+}
+
 qlora_status linear_forward(const qlora_nf4& W, const LevelTable& t, const void* A,
                             const void* B, int32_t r, float alpha, const void* X, int64_t M,
-                            void* Y, float* U_save, void* workspace, cudaStream_t s) {
+                            void* Y, float* U_save, void* workspace, cudaStream_t s,
+                            const LoraOpts& o) {
   const int64_t N = W.rows, K = W.cols;
   const QView w = view_of(W);
   char* ws = static_cast<char*>(workspace);
   auto* st = reinterpret_cast<DeviceStatus*>(ws);
-  const float sc = lora_scale(alpha, r);
+  const float sc = lora_scale(alpha, o.r_adapter);
+  const int32_t* seg = o.seg;
+  const int32_t r_adapter = o.r_adapter;
+  if ((seg || o.mask) && !linear_multi_supported(M, N, K, r)) return QLORA_ERR_UNSUPPORTED;
+  // the adapter branch's input: X, or its dropped-out copy X (.) D
+  const void* xl = X;
+  if (o.mask) {
+    QLORA_TRY(dropout_apply(X, o.mask, M, K, const_cast<void*>(o.x_drop), s));
+    xl = o.x_drop;
+  }
   if (use_tc(M, N, K, r) && use_small(M)) {
     const SmallLayout L = small_layout(M, N, K, r);
     const int32_t r16 = lora_rows(r), span = lora_span(r);
     char* su = ws + L.su;
     float* part = reinterpret_cast<float*>(ws + L.part_f);
-    QLORA_TRY(small_down_partial(X, A, static_cast<int>(M), K, r, part, s));
+    QLORA_TRY(small_down_partial(xl, A, static_cast<int>(M), K, r, part, s));
     ReduceArgs ra = reduce_args(part, small_chunks(K), M, r, r16);
+    ra.seg = seg;  // U / V: each token keeps only its adapter's columns
+    ra.seg_cols = r_adapter;
     ra.o1 = U_save;
     ra.ld1 = r;
-    ra.a1 = 1.0f;
+    ra.a1 = o.keep;
     ra.o2 = su;
     ra.ld2 = 2 * span;
-    ra.a2 = sc;
+    ra.a2 = sc * o.keep;
     ra.o2_lo = span;
     ra.o2_pad = 1;  // the padding columns meet zero B columns in the MMA: written as zeros
     QLORA_TRY(splitk_reduce(ra, s));
@@ -219,14 +236,16 @@ qlora_status linear_forward(const qlora_nf4& W, const LevelTable& t, const void*
     char* su = ws + L.su;
     float* part = reinterpret_cast<float*>(ws + L.part_f);
     // U = X A^T (split-K over d_in) -> U_save (fp32) and sU = s U as bf16 hi + lo
-    QLORA_TRY(tc_lora_gemm(X, false, M, K, K, A, K, r, r16, part, sp.u, st, s));
+    QLORA_TRY(tc_lora_gemm(xl, false, M, K, K, A, K, r, r16, part, sp.u, st, s));
     ReduceArgs ra = reduce_args(part, sp.u, M, r, r16);
+    ra.seg = seg;  // U / V: each token keeps only its adapter's columns
+    ra.seg_cols = r_adapter;
     ra.o1 = U_save;
     ra.ld1 = r;
-    ra.a1 = 1.0f;
+    ra.a1 = o.keep;
     ra.o2 = su;
     ra.ld2 = 2 * span;
-    ra.a2 = sc;
+    ra.a2 = sc * o.keep;
     ra.o2_lo = span;
     ra.o2_pad = 1;  // the padding columns meet zero B columns in the MMA: written as zeros
     QLORA_TRY(splitk_reduce(ra, s));
@@ -260,9 +279,18 @@ qlora_status linear_forward(const qlora_nf4& W, const LevelTable& t, const void*
 qlora_status linear_backward(const qlora_nf4& W, const LevelTable& t, const void* A,
                              const void* B, int32_t r, float alpha, const void* X,
                              const float* U, const void* dY, int64_t M, void* dX, float* dA,
-                             float* dB, bool accumulate, void* workspace, cudaStream_t s) {
+                             float* dB, bool accumulate, void* workspace, cudaStream_t s,
+                             const LoraOpts& o) {
   const int64_t N = W.rows, K = W.cols;
-  const float sc = lora_scale(alpha, r);
+  const float sc = lora_scale(alpha, o.r_adapter);
+  const int32_t* seg = o.seg;
+  const int32_t r_adapter = o.r_adapter;
+  if ((seg || o.mask) && !linear_multi_supported(M, N, K, r)) return QLORA_ERR_UNSUPPORTED;
+  // with dropout the adapter branch saw X (.) D: dA and a recomputed U read it,
+  // the LoRA stage of the dX GEMM is switched off (sV = 0) and the masked
+  // term D (.) s V A / (1 - p) is added to dX afterwards
+  const void* xl = o.mask ? o.x_drop : X;
+  const float sc_dx = o.mask ? 0.0f : sc;
   const QView w = view_of(W);
   char* ws = static_cast<char*>(workspace);
   auto* st = reinterpret_cast<DeviceStatus*>(ws);
@@ -278,13 +306,15 @@ qlora_status linear_backward(const qlora_nf4& W, const LevelTable& t, const void
     QLORA_TRY(small_v_partial(dY, B, m, N, r, part, s));
     {
       ReduceArgs ra = reduce_args(part, small_chunks(N), M, r, r16);
+      ra.seg = seg;  // U / V: each token keeps only its adapter's columns
+      ra.seg_cols = r_adapter;
       ra.o1 = v;
       ra.ld1 = r;
       ra.a1 = 1.0f;
       if (!gemv) {
         ra.o2 = sv;
         ra.ld2 = 2 * span;
-        ra.a2 = sc;
+        ra.a2 = sc_dx;
         ra.o2_lo = span;
         ra.o2_pad = 1;
       }
@@ -292,18 +322,20 @@ qlora_status linear_backward(const qlora_nf4& W, const LevelTable& t, const void
     }
     if (!U) {
       float* u = reinterpret_cast<float*>(ws + L.u);
-      QLORA_TRY(small_down_partial(X, A, m, K, r, part, s));
+      QLORA_TRY(small_down_partial(xl, A, m, K, r, part, s));
       ReduceArgs ra = reduce_args(part, small_chunks(K), M, r, r16);
+      ra.seg = seg;  // U / V: each token keeps only its adapter's columns
+      ra.seg_cols = r_adapter;
       ra.o1 = u;
       ra.ld1 = r;
-      ra.a1 = 1.0f;
+      ra.a1 = o.keep;
       QLORA_TRY(splitk_reduce(ra, s));
       U = u;
     }
     if (dX && gemv) {
       // dX = dY W + s V A: CTA partials of the dequant GEMV, summed in order
       float* fpart = reinterpret_cast<float*>(ws + L.fused_b);
-      QLORA_TRY(gemv_dgrad(w, t, dY, M, v, A, r, sc, fpart, s));
+      QLORA_TRY(gemv_dgrad(w, t, dY, M, v, A, r, sc_dx, fpart, s));
       ReduceArgs rx = reduce_args(fpart, gemv_dgrad_chunks(M, K), M, static_cast<int>(K),
                                   static_cast<int>(K));
       rx.o2 = dX;
@@ -324,8 +356,9 @@ qlora_status linear_backward(const qlora_nf4& W, const LevelTable& t, const void
         QLORA_TRY(splitk_reduce(rx, s));
       }
     }
+    if (dX && o.mask) QLORA_TRY(dropout_dx(dX, v, r, A, o.mask, M, K, r, sc * o.keep, s));
     QLORA_TRY(small_grad_b(dY, U, m, N, r, sc, accumulate, dB, s));
-    return small_grad_a(v, X, m, K, r, sc, accumulate, dA, s);
+    return small_grad_a(v, xl, m, K, r, sc * o.keep, accumulate, dA, s);
   }
   if (use_tc(M, N, K, r)) {
     const TcLayout L = tc_layout(M, N, K, r);
@@ -343,11 +376,18 @@ qlora_status linear_backward(const qlora_nf4& W, const LevelTable& t, const void
     QLORA_TRY(tc_lora_gemm(dY, false, M, N, N, bt, N, r, r16, part, sp.v, st, s));
     {
       ReduceArgs ra = reduce_args(part, sp.v, M, r, r16);
+      ra.seg = seg;  // U / V: each token keeps only its adapter's columns
+      ra.seg_cols = r_adapter;
       ra.o2 = sv;
       ra.ld2 = 2 * span;
-      ra.a2 = sc;
+      ra.a2 = sc_dx;
       ra.o2_lo = span;
       ra.o2_pad = 1;
+      if (o.mask) {
+        ra.o1 = reinterpret_cast<float*>(ws + L.v32);
+        ra.ld1 = r;
+        ra.a1 = 1.0f;
+      }
       ra.o3 = vt;
       ra.ld3 = mp;
       ra.a3 = 1.0f;
@@ -367,11 +407,13 @@ qlora_status linear_backward(const qlora_nf4& W, const LevelTable& t, const void
       if (U) {
         QLORA_TRY(transpose_to_bf16(U, true, M, r, r, ut, mp, r16, s2));
       } else {
-        QLORA_TRY(tc_lora_gemm(X, false, M, K, K, A, K, r, r16, part, sp.u, st, s2));
+        QLORA_TRY(tc_lora_gemm(xl, false, M, K, K, A, K, r, r16, part, sp.u, st, s2));
         ReduceArgs ra = reduce_args(part, sp.u, M, r, r16);
+        ra.seg = seg;  // U / V: each token keeps only its adapter's columns
+        ra.seg_cols = r_adapter;
         ra.o3 = ut;
         ra.ld3 = mp;
-        ra.a3 = 1.0f;
+        ra.a3 = o.keep;
         ra.o3_lo = r16;
         QLORA_TRY(splitk_reduce(ra, s2));
       }
@@ -387,13 +429,13 @@ qlora_status linear_backward(const qlora_nf4& W, const LevelTable& t, const void
         QLORA_TRY(splitk_reduce(ra, s2));
       }
       // dA = s V^T X: rows d_in, stored transposed as r x d_in
-      QLORA_TRY(tc_lora_gemm(X, true, K, M, K, vt, mp, 2 * r16, 2 * r16, part, sp.da, st, s2));
+      QLORA_TRY(tc_lora_gemm(xl, true, K, M, K, vt, mp, 2 * r16, 2 * r16, part, sp.da, st, s2));
       ReduceArgs ra = reduce_args(part, sp.da, K, r, 2 * r16);
       ra.lo = r16;
       ra.o1 = dA;
       ra.ld1 = K;
       ra.trans1 = true;
-      ra.a1 = sc;
+      ra.a1 = sc * o.keep;
       ra.acc1 = accumulate;
       return splitk_reduce(ra, s2);
     };
@@ -401,14 +443,20 @@ qlora_status linear_backward(const qlora_nf4& W, const LevelTable& t, const void
       // dX = dY W + sV A in one kernel (split over d_out when needed)
       if (!dX) return QLORA_OK;
       const FusedShape f = fused_shape(M, K, ceil_div(N, 64));
-      if (f.splits == 1) return tc_fused_dgrad(w, t, dY, M, sv, A, r, dX, f, st, s);
-      float* fpart = reinterpret_cast<float*>(ws + L.fused_b);
-      QLORA_TRY(tc_fused_dgrad(w, t, dY, M, sv, A, r, fpart, f, st, s));
-      ReduceArgs rx = reduce_args(fpart, f.splits, M, static_cast<int>(K), static_cast<int>(K));
-      rx.o2 = dX;
-      rx.ld2 = K;
-      rx.a2 = 1.0f;
-      return splitk_reduce(rx, s);
+      if (f.splits == 1) {
+        QLORA_TRY(tc_fused_dgrad(w, t, dY, M, sv, A, r, dX, f, st, s));
+      } else {
+        float* fpart = reinterpret_cast<float*>(ws + L.fused_b);
+        QLORA_TRY(tc_fused_dgrad(w, t, dY, M, sv, A, r, fpart, f, st, s));
+        ReduceArgs rx = reduce_args(fpart, f.splits, M, static_cast<int>(K), static_cast<int>(K));
+        rx.o2 = dX;
+        rx.ld2 = K;
+        rx.a2 = 1.0f;
+        QLORA_TRY(splitk_reduce(rx, s));
+      }
+      if (!o.mask) return QLORA_OK;
+      return dropout_dx(dX, reinterpret_cast<const float*>(ws + L.v32), r, A, o.mask, M, K, r,
+                        sc * o.keep, s);
     };
     // the fused kernel is enqueued first so that its first wave takes the SMs
     const qlora_status st_main = main_work();

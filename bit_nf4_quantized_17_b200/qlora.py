@@ -51,6 +51,14 @@ class qlora_nf4(ctypes.Structure):
     ]
 
 
+class qlora_adapter_opts(ctypes.Structure):
+    _fields_ = [
+        ("n_adapters", ctypes.c_int32), ("reserved", ctypes.c_int32),
+        ("adapter", ctypes.c_void_p), ("dropout_p", ctypes.c_float),
+        ("reserved2", ctypes.c_int32), ("keep_mask", ctypes.c_void_p), ("x_drop", ctypes.c_void_p),
+    ]
+
+
 class QloraError(RuntimeError):
     def __init__(self, status, where):
         self.status = int(status)
@@ -72,6 +80,7 @@ def lib():
                                  ctypes.c_void_p, ctypes.c_float)
         psz = ctypes.POINTER(ctypes.c_size_t)
         pq = ctypes.POINTER(qlora_nf4)
+        po = ctypes.POINTER(qlora_adapter_opts)
         sig = {
             "qlora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
             "qlora_levels": (ctypes.c_int, [i32, ctypes.POINTER(ctypes.c_float)]),
@@ -82,6 +91,14 @@ def lib():
             "qlora_linear_fwd": (ctypes.c_int, [pq, vp, vp, i32, f32, vp, i64, vp, vp, vp, sz, vp]),
             "qlora_linear_bwd": (ctypes.c_int, [pq, vp, vp, i32, f32, vp, vp, vp, i64, vp, vp, vp,
                                                 i32, vp, sz, vp]),
+            "qlora_linear_fwd_multi": (ctypes.c_int, [pq, vp, vp, i32, i32, f32, vp, vp, i64, vp,
+                                                      vp, vp, sz, vp]),
+            "qlora_linear_bwd_multi": (ctypes.c_int, [pq, vp, vp, i32, i32, f32, vp, vp, vp, vp,
+                                                      i64, vp, vp, vp, i32, vp, sz, vp]),
+            "qlora_linear_fwd_ex": (ctypes.c_int, [pq, vp, vp, i32, f32, po, vp, i64, vp, vp, vp,
+                                                   sz, vp]),
+            "qlora_linear_bwd_ex": (ctypes.c_int, [pq, vp, vp, i32, f32, po, vp, vp, vp, i64, vp,
+                                                   vp, vp, i32, vp, sz, vp]),
             "qlora_check": (ctypes.c_int, [vp, vp]),
             "qlora_merge": (ctypes.c_int, [pq, vp, vp, i32, f32, vp, vp]),
             "qlora_paged_alloc": (ctypes.c_int, [ctypes.c_size_t, ctypes.POINTER(ctypes.c_void_p)]),
@@ -223,6 +240,131 @@ def qlora_linear_fwd(q, A, B, alpha, X, Y=None, U_save=None, workspace=None, str
     if check:
         qlora_check(workspace, stream)
     return Y
+
+
+def qlora_linear_fwd_multi(q, A, B, r, alpha, adapter, X, Y=None, U_save=None, workspace=None,
+                           stream=None, check=False):
+    """Several rank-r adapters stacked along the rank (A: (n r) x d_in, B:
+    d_out x (n r)); token m uses adapter adapter[m] (int32, -1 = none)."""
+    M = X.shape[0]
+    rt = A.shape[0]
+    if rt % r:
+        raise ValueError(f"A has {rt} rows: not a stack of rank-{r} adapters")
+    n = rt // r
+    assert adapter.dtype == torch.int32 and adapter.numel() == M
+    if Y is None:
+        Y = torch.empty((M, q.rows), dtype=torch.bfloat16, device=X.device)
+    if workspace is None:
+        workspace = _workspace(qlora_linear_workspace(M, q.rows, q.cols, rt)[0], X.device)
+    st = q.struct
+    _ok(lib().qlora_linear_fwd_multi(ctypes.byref(st), _ptr(A), _ptr(B), n, r, float(alpha),
+                                     _ptr(adapter), _ptr(X), M, _ptr(Y), _ptr(U_save),
+                                     _ptr(workspace), workspace.numel(), _stream(stream)),
+        "qlora_linear_fwd_multi")
+    if check:
+        qlora_check(workspace, stream)
+    return Y
+
+
+def qlora_linear_bwd_multi(q, A, B, r, alpha, adapter, X, U, dY, dX=None, dA=None, dB=None,
+                           accumulate=False, want_dx=True, workspace=None, stream=None,
+                           check=False):
+    """Backward of qlora_linear_fwd_multi; dA and dB in the stacked layouts."""
+    M = X.shape[0]
+    rt = A.shape[0]
+    if rt % r:
+        raise ValueError(f"A has {rt} rows: not a stack of rank-{r} adapters")
+    n = rt // r
+    dev = X.device
+    assert adapter.dtype == torch.int32 and adapter.numel() == M
+    if want_dx and dX is None:
+        dX = torch.empty((M, q.cols), dtype=torch.bfloat16, device=dev)
+    if dA is None:
+        dA = torch.empty((rt, q.cols), dtype=torch.float32, device=dev)
+    if dB is None:
+        dB = torch.empty((q.rows, rt), dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = _workspace(qlora_linear_workspace(M, q.rows, q.cols, rt)[1], dev)
+    st = q.struct
+    _ok(lib().qlora_linear_bwd_multi(ctypes.byref(st), _ptr(A), _ptr(B), n, r, float(alpha),
+                                     _ptr(adapter), _ptr(X), _ptr(U), _ptr(dY), M,
+                                     _ptr(dX) if want_dx else None, _ptr(dA), _ptr(dB),
+                                     1 if accumulate else 0, _ptr(workspace), workspace.numel(),
+                                     _stream(stream)), "qlora_linear_bwd_multi")
+    if check:
+        qlora_check(workspace, stream)
+    return dX, dA, dB
+
+
+def dropout_keep_mask(M, K, p, generator=None, device="cuda"):
+    """A keep mask for LoRA dropout, drawn with torch's generator (the random
+    draw is an input of the layer): M x K/8 uint8, bit (k % 8) of byte
+    [m][k / 8] set = keep X[m][k], each kept with probability 1 - p."""
+    keep = torch.rand((M, K // 8, 8), generator=generator, device=device) >= p
+    weights = (1 << torch.arange(8, device=device, dtype=torch.int32))
+    return (keep.to(torch.int32) * weights).sum(-1).to(torch.uint8).contiguous()
+
+
+def _opts(r, A, adapter, p, keep_mask, x_drop):
+    o = qlora_adapter_opts()
+    rt = A.shape[0]
+    if rt % r:
+        raise ValueError(f"A has {rt} rows: not a stack of rank-{r} adapters")
+    o.n_adapters = rt // r
+    o.adapter = adapter.data_ptr() if adapter is not None else None
+    o.dropout_p = float(p)
+    o.keep_mask = keep_mask.data_ptr() if keep_mask is not None else None
+    o.x_drop = x_drop.data_ptr() if x_drop is not None else None
+    return o
+
+
+def qlora_linear_fwd_ex(q, A, B, r, alpha, X, adapter=None, p=0.0, keep_mask=None, x_drop=None,
+                        Y=None, U_save=None, workspace=None, stream=None, check=False):
+    """Forward with optional per-token adapters (A, B stacked along the rank)
+    and LoRA dropout (keep_mask from dropout_keep_mask; x_drop receives
+    X (.) D and must be passed again to the backward)."""
+    M = X.shape[0]
+    rt = A.shape[0]
+    o = _opts(r, A, adapter, p, keep_mask, x_drop)
+    if Y is None:
+        Y = torch.empty((M, q.rows), dtype=torch.bfloat16, device=X.device)
+    if workspace is None:
+        workspace = _workspace(qlora_linear_workspace(M, q.rows, q.cols, rt)[0], X.device)
+    st = q.struct
+    _ok(lib().qlora_linear_fwd_ex(ctypes.byref(st), _ptr(A), _ptr(B), r, float(alpha),
+                                  ctypes.byref(o), _ptr(X), M, _ptr(Y), _ptr(U_save),
+                                  _ptr(workspace), workspace.numel(), _stream(stream)),
+        "qlora_linear_fwd_ex")
+    if check:
+        qlora_check(workspace, stream)
+    return Y
+
+
+def qlora_linear_bwd_ex(q, A, B, r, alpha, X, U, dY, adapter=None, p=0.0, keep_mask=None,
+                        x_drop=None, dX=None, dA=None, dB=None, accumulate=False, want_dx=True,
+                        workspace=None, stream=None, check=False):
+    """Backward of qlora_linear_fwd_ex (same adapter ids, mask and x_drop)."""
+    M = X.shape[0]
+    rt = A.shape[0]
+    dev = X.device
+    o = _opts(r, A, adapter, p, keep_mask, x_drop)
+    if want_dx and dX is None:
+        dX = torch.empty((M, q.cols), dtype=torch.bfloat16, device=dev)
+    if dA is None:
+        dA = torch.empty((rt, q.cols), dtype=torch.float32, device=dev)
+    if dB is None:
+        dB = torch.empty((q.rows, rt), dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = _workspace(qlora_linear_workspace(M, q.rows, q.cols, rt)[1], dev)
+    st = q.struct
+    _ok(lib().qlora_linear_bwd_ex(ctypes.byref(st), _ptr(A), _ptr(B), r, float(alpha),
+                                  ctypes.byref(o), _ptr(X), _ptr(U), _ptr(dY), M,
+                                  _ptr(dX) if want_dx else None, _ptr(dA), _ptr(dB),
+                                  1 if accumulate else 0, _ptr(workspace), workspace.numel(),
+                                  _stream(stream)), "qlora_linear_bwd_ex")
+    if check:
+        qlora_check(workspace, stream)
+    return dX, dA, dB
 
 
 def qlora_linear_bwd(q, A, B, alpha, X, U, dY, dX=None, dA=None, dB=None, accumulate=False,

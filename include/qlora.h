@@ -170,6 +170,35 @@ qlora_status qlora_linear_bwd(const qlora_nf4* W, const void* A, const void* B,
                               float* dB, int32_t accumulate, void* workspace,
                               size_t workspace_bytes, void* stream);
 
+/* Several adapters over one quantised base ("LoRA 与 QLoRA：把大模型微调拆成
+ * 可负担的工程", section 3: one base, one small adapter per task, switched per
+ * request).  n_adapters adapters of rank r share W; token m uses adapter
+ * adapter[m] (device int32; an id outside [0, n_adapters), e.g. -1, selects
+ * none: that token gets the base output only).  With a = adapter[m]:
+ *     Y[m]  = X[m] W^T + s (X[m] A_a^T) B_a^T,           s = alpha / r
+ *     dX[m] = dY[m] W + s (dY[m] B_a) A_a
+ *     dA_a  = s sum_{m: a} (dY[m] B_a)^T X[m],  dB_a = s sum_{m: a} dY[m]^T (X[m] A_a^T)
+ * The adapters are stacked along the rank: A is (n_adapters r) x K bf16 with
+ * A_a in rows [a r, (a+1) r); B is N x (n_adapters r) bf16 with B_a in
+ * columns [a r, (a+1) r); dA and dB (fp32) have the same layouts and U_save /
+ * U are M x (n_adapters r) fp32 holding X[m] A_a^T in the token's own
+ * columns and zeros elsewhere.  Workspace sizes: qlora_linear_workspace with
+ * rank n_adapters * r.  Requirements as qlora_linear_fwd / _bwd, plus
+ * n_adapters >= 1, n_adapters * r <= 256, and N and n_adapters * r multiples
+ * of 8 (else QLORA_ERR_UNSUPPORTED); `adapter` 4-byte aligned, NULL only
+ * when M = 0. */
+qlora_status qlora_linear_fwd_multi(const qlora_nf4* W, const void* A, const void* B,
+                                    int32_t n_adapters, int32_t r, float alpha,
+                                    const int32_t* adapter, const void* X, int64_t M, void* Y,
+                                    float* U_save, void* workspace, size_t workspace_bytes,
+                                    void* stream);
+qlora_status qlora_linear_bwd_multi(const qlora_nf4* W, const void* A, const void* B,
+                                    int32_t n_adapters, int32_t r, float alpha,
+                                    const int32_t* adapter, const void* X, const float* U,
+                                    const void* dY, int64_t M, void* dX, float* dA, float* dB,
+                                    int32_t accumulate, void* workspace,
+                                    size_t workspace_bytes, void* stream);
+
 /* Merge a trained adapter into a restored 16-bit weight ("LoRA 与 QLoRA：把
  * 大模型微调拆成可负担的工程", section 3: after training B A has the shape of
  * W and is added to it; 4-bit storage cannot take the update):
@@ -198,6 +227,45 @@ qlora_status qlora_merge(const qlora_nf4* W, const void* A, const void* B, int32
 qlora_status qlora_adamw(float* param, void* param_bf16, const float* grad, float* m, float* v,
                          int64_t n, int32_t step, float lr, float beta1, float beta2, float eps,
                          float weight_decay, float grad_scale, void* stream);
+
+/* The general form of the two calls above, with LoRA dropout on the adapter
+ * input ("LoRA 与 QLoRA：把大模型微调拆成可负担的工程", section 4.3,
+ * lora_dropout; "QLoRA 量化微调", training recipe).  The adapter branch reads
+ * X~ = D (.) X / (1 - p) for a keep mask D that the caller draws, the base
+ * branch reads X:
+ *     Y  = X W^T + s U B^T,               U = X~ A^T   (U_save / U hold this U)
+ *     dX = dY W + s D (.) (V A) / (1 - p),  dA = s V^T X~,  dB = s dY^T U
+ * Fields of qlora_adapter_opts:
+ *   n_adapters, adapter  as for the *_multi calls (n_adapters = 1 and
+ *                        adapter = NULL: one adapter for every token);
+ *   dropout_p            p in [0, 1); keep_mask = NULL turns dropout off;
+ *   keep_mask            device, M x K/8 bytes: bit (k % 8) of byte
+ *                        m K/8 + k/8 set = keep X[m][k];
+ *   x_drop               device, M x K bf16, 16-byte aligned: written by the
+ *                        forward with D (.) X (kept values, unscaled), read
+ *                        by the backward (pass the same buffer and mask).
+ * Dropout needs the same conditions as several adapters (N and the stacked
+ * rank multiples of 8, else QLORA_ERR_UNSUPPORTED).  Errors as the *_multi
+ * calls, plus QLORA_ERR_UNSUPPORTED for p outside [0, 1) and QLORA_ERR_NULL
+ * for a mask without x_drop. */
+typedef struct {
+  int32_t n_adapters;
+  int32_t reserved;
+  const int32_t* adapter;
+  float dropout_p;
+  int32_t reserved2;
+  const uint8_t* keep_mask;
+  void* x_drop;
+} qlora_adapter_opts;
+qlora_status qlora_linear_fwd_ex(const qlora_nf4* W, const void* A, const void* B, int32_t r,
+                                 float alpha, const qlora_adapter_opts* opts, const void* X,
+                                 int64_t M, void* Y, float* U_save, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+qlora_status qlora_linear_bwd_ex(const qlora_nf4* W, const void* A, const void* B, int32_t r,
+                                 float alpha, const qlora_adapter_opts* opts, const void* X,
+                                 const float* U, const void* dY, int64_t M, void* dX, float* dA,
+                                 float* dB, int32_t accumulate, void* workspace,
+                                 size_t workspace_bytes, void* stream);
 
 /* Paged optimiser states.  The optimiser moments can live in CUDA managed
  * (unified) memory, which the driver migrates between host and device pages

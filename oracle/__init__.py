@@ -21,6 +21,11 @@ What it computes, and where the method is stated:
   section 3).
 * ``optim.py`` - the AdamW step for the adapters (the optimiser that updates
   only A and B, "QLoRA技术从入门到精通", section 3(3)).
+* ``multi.py`` - several adapters over one base, one per token ("LoRA 与
+  QLoRA：把大模型微调拆成可负担的工程", section 3: shared base, one small pair
+  per task).
+* ``dropout.py`` - LoRA dropout on the adapter input, with the keep mask as an
+  input ("LoRA 与 QLoRA：把大模型微调拆成可负担的工程", section 4.3).
 * ``bf16.py``  - the bf16 <-> fp32 conversions; the products use the
   dequantised weight rounded to bf16 (``compute_weight``), the compute dtype
   the pages name.
@@ -55,6 +60,8 @@ from .nf4 import (
 )
 from .linear import lora_scale, linear_fwd, linear_bwd, merge_weight
 from .optim import adamw_step
+from .multi import linear_fwd_multi, linear_bwd_multi
+from .dropout import unpack_keep_mask, linear_fwd_dropout, linear_bwd_dropout
 
 __all__ = [
     "bf16_bits_to_f32", "f32_to_bf16_bits", "round_to_bf16",
@@ -62,4 +69,6 @@ __all__ = [
     "block_absmax", "pack_nibbles", "unpack_nibbles", "fixed_point_mean",
     "double_quantize", "dequantize_scales", "block_scales", "quantize", "dequantize", "compute_weight",
     "storage_bits", "lora_scale", "linear_fwd", "linear_bwd", "merge_weight", "adamw_step",
+    "linear_fwd_multi", "linear_bwd_multi", "unpack_keep_mask", "linear_fwd_dropout",
+    "linear_bwd_dropout",
 ]

@@ -173,3 +173,21 @@ def test_adamw_and_paged_argument_errors_without_cuda():
     assert L.qlora_paged_prefetch(None, 64, 1, None) == Q.QLORA_ERR_NULL
     assert L.qlora_paged_prefetch(a, 0, 1, None) == Q.QLORA_ERR_SHAPE
     assert L.qlora_paged_free(None) == Q.QLORA_OK
+
+
+def test_multi_adapter_argument_errors_without_cuda():
+    L = Q.lib()
+    q = _fake_q(256, 256)
+    P = ctypes.c_void_p
+    ws = Q.qlora_linear_workspace(4, 256, 256, 32)[0]
+
+    def fwd(n=4, r=8, ids=P(0x50000), M=4):
+        return L.qlora_linear_fwd_multi(ctypes.byref(q), P(0x100000), P(0x110000), n, r, 8.0, ids,
+                                        P(0x120000), M, P(0x130000), None, P(0x140000), ws, None)
+
+    assert fwd(n=0) == Q.QLORA_ERR_SHAPE
+    assert fwd(n=33) == Q.QLORA_ERR_SHAPE          # 264 stacked ranks
+    assert fwd(ids=None) == Q.QLORA_ERR_NULL
+    assert fwd(ids=P(0x50002)) == Q.QLORA_ERR_ALIGN
+    assert fwd(n=3, r=5) == Q.QLORA_ERR_UNSUPPORTED  # 15 stacked ranks
+    assert fwd(M=0, ids=None) == Q.QLORA_OK          # nothing to do: no launch

@@ -114,25 +114,26 @@ def test_paged_states_match_device_states():
 
 
 def test_training_step_moves_adapters_downhill():
-    # forward, backward and AdamW on one layer: the loss 0.5 |Y - T|^2 falls
+    # forward, backward and AdamW on one layer, B starting at zero, towards
+    # the output of the same layer with another B: 0.5 |Y - T|^2 falls
     from bit_nf4_quantized_17_b200 import workloads as WL
     shape = WL.LinearShape(512, 1024, 16, 32.0)
     inp = WL.linear_inputs(shape, 256, 11)
     q = Q.qlora_quantize(inp["W"].to(DEV))
     X = inp["X"].to(DEV)
-    B0 = WL.randn((512, 16), 0.02, 3, torch.bfloat16).to(DEV)
-    opt = AdapterAdamW(inp["A"].to(DEV), B0, lr=2e-3)
-    T = (Q.qlora_linear_fwd(q, opt.A, opt.B, shape.alpha, X).float()
-         + 0.5 * torch.randn(256, 512, device=DEV)).to(torch.bfloat16)
+    A0 = inp["A"].to(DEV)
+    B_target = WL.randn((512, 16), 0.05, 4, torch.bfloat16).to(DEV)
+    T = Q.qlora_linear_fwd(q, A0, B_target, shape.alpha, X).float()
+    opt = AdapterAdamW(A0, torch.zeros_like(B_target), lr=5e-3)
     bucket = opt.grad_bucket()
     U = torch.empty((256, 16), dtype=torch.float32, device=DEV)
     losses = []
-    for _ in range(20):
+    for _ in range(30):
         Y = Q.qlora_linear_fwd(q, opt.A, opt.B, shape.alpha, X, U_save=U)
-        dY = (Y.float() - T.float())
+        dY = Y.float() - T
         losses.append(0.5 * float((dY * dY).sum()))
         Q.qlora_linear_bwd(q, opt.A, opt.B, shape.alpha, X, U, dY.to(torch.bfloat16),
                            dA=bucket.dA, dB=bucket.dB, want_dx=False)
         opt.step(bucket)
     torch.cuda.synchronize()
-    assert losses[-1] < 0.9 * losses[0], losses
+    assert losses[-1] < 0.2 * losses[0], losses

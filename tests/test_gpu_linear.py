@@ -202,3 +202,47 @@ def test_zero_tokens():
                                                             device=DEV), dA=dA, dB=dB)
     torch.cuda.synchronize()
     assert torch.count_nonzero(dA) == 0 and torch.count_nonzero(dB) == 0
+
+
+@pytest.mark.parametrize("M", [1, 2, 16, 700, 4096])
+def test_cuda_graph_replay_matches_eager(M):
+    # forward and backward captured in CUDA graphs (the backward forks onto a
+    # second stream and joins back inside the graph) give the eager results
+    # bit for bit, replay after replay
+    shape = WL.LinearShape(1024, 2048, 16, 32.0)
+    inp = WL.linear_inputs(shape, M, 900 + M)
+    q = Q.qlora_quantize(inp["W"].to(DEV))
+    A, B, X, dY = (inp[k].to(DEV) for k in ("A", "B", "X", "dY"))
+    fb, bb = Q.qlora_linear_workspace(M, shape.d_out, shape.d_in, shape.r)
+    fws = torch.zeros(fb, dtype=torch.uint8, device=DEV)
+    bws = torch.zeros(bb, dtype=torch.uint8, device=DEV)
+    Y = torch.empty((M, shape.d_out), dtype=torch.bfloat16, device=DEV)
+    U = torch.empty((M, shape.r), dtype=torch.float32, device=DEV)
+    dX = torch.empty((M, shape.d_in), dtype=torch.bfloat16, device=DEV)
+    dA = torch.empty((shape.r, shape.d_in), dtype=torch.float32, device=DEV)
+    dB = torch.empty((shape.d_out, shape.r), dtype=torch.float32, device=DEV)
+
+    def step():
+        Q.qlora_linear_fwd(q, A, B, shape.alpha, X, Y=Y, U_save=U, workspace=fws)
+        Q.qlora_linear_bwd(q, A, B, shape.alpha, X, U, dY, dX=dX, dA=dA, dB=dB, workspace=bws)
+
+    step()
+    torch.cuda.synchronize()
+    ref = [t.clone() for t in (Y, U, dX, dA, dB)]
+    g = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream()
+    cap.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(g, stream=cap):
+            step()
+    torch.cuda.current_stream().wait_stream(cap)
+    for t in (Y, U, dX, dA, dB):
+        t.zero_()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    for a, b in zip((Y, U, dX, dA, dB), ref):
+        assert torch.equal(a, b)
+    Q.qlora_check(fws)
+    Q.qlora_check(bws)
+    del g
