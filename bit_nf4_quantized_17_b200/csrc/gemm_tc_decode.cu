@@ -33,14 +33,16 @@ using tc::block_tables;
 using tc::expand8;
 
 constexpr int kThreads = 320;
-constexpr int kStages = 4;
+constexpr int kStages = 8;  // shared-memory stages (TMA in flight)
+constexpr int kSlots = 4;   // TMEM slots for the dequantised W of a k-tile
 constexpr int kXBytes = 2048;                    // 16 token rows x 64 bf16 (128B swizzle)
 constexpr int kCodeBytes = 4096;                 // 128 W rows x 32 bytes
 constexpr int kStageBytes = kXBytes + kCodeBytes;
 constexpr int kExtABytes = 16384;                // 128 rows of B x 64 ranks
 constexpr int kExtBBytes = 2048;                 // 16 tokens x 64 ranks of [hi | lo]
-constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kExtABytes + kExtBBytes + 256;
-constexpr uint32_t kTmemCols = 256;              // D: [0, 16); A stage s: [32 + 32 s, 64 + 32 s)
+constexpr int kRedBytes = 16 * 128 * 4;          // this CTA's fp32 output tile (cluster reduce)
+constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kExtABytes + kExtBBytes + kRedBytes + 256;
+constexpr uint32_t kTmemCols = 256;              // D: [0, 16); A slot a: [32 + 32 a, 64 + 32 a)
 constexpr long long kTimeoutCycles = 4000000000ll;
 
 struct DecArgs {
@@ -50,9 +52,9 @@ struct DecArgs {
   QView w;
   int32_t kblocks;
   int64_t nblocks;
-  void* out;
-  int32_t out_bf16;
-  int64_t split_stride, out_elems;
+  __nv_bfloat16* out;  // Y, M x N
+  int64_t out_elems;
+  int32_t cluster;  // > 1: the splits of a row tile form a cluster and sum in shared memory
   DeviceStatus* st;
 };
 
@@ -89,13 +91,15 @@ tc_decode_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  // [kStages x (X | codes)] [ext A | ext B] [barriers]
+  // [kStages x (X | codes)] [ext A | ext B] [output tile] [barriers]
   uint8_t* ext_a = smem + kStages * kStageBytes;
   uint8_t* ext_b = ext_a + kExtABytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(ext_b + kExtBBytes);
-  uint64_t* afull = full + kStages;  // the stage's W rows are in TMEM
-  uint64_t* empty = afull + kStages; // the stage's MMAs are done
-  uint64_t* ext_full = empty + kStages;
+  float* red = reinterpret_cast<float*>(ext_b + kExtBBytes);  // [16 tokens][128 rows]
+  uint64_t* full = reinterpret_cast<uint64_t*>(ext_b + kExtBBytes + kRedBytes);
+  uint64_t* empty = full + kStages;   // the stage's MMAs are done
+  uint64_t* afull = empty + kStages;  // the slot holds the k-tile's W rows
+  uint64_t* aempty = afull + kSlots;  // the slot's MMAs are done
+  uint64_t* ext_full = aempty + kSlots;
   uint64_t* ext_empty = ext_full + 1;
   uint64_t* accum = ext_empty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
@@ -110,8 +114,11 @@ tc_decode_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       ptx::mbar_init(&full[s], 1);
-      ptx::mbar_init(&afull[s], 4);  // the four warps of the group
       ptx::mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < kSlots; ++a) {
+      ptx::mbar_init(&afull[a], 4);  // the four warps of the group
+      ptx::mbar_init(&aempty[a], 1);
     }
     ptx::mbar_init(ext_full, 1);
     ptx::mbar_init(ext_empty, 1);
@@ -170,10 +177,10 @@ tc_decode_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
     const uint32_t idesc = ptx::idesc_bf16(128, 16, 0, 0);
     bool ok = true;
     for (int i = 0; i < kn && ok; ++i) {
-      const int s = i % kStages;
-      const uint32_t ph = (i / kStages) & 1;
+      const int s = i % kStages, a = i % kSlots;
+      const uint32_t ph = (i / kStages) & 1, pa = (i / kSlots) & 1;
       if (!ptx::mbar_wait(&full[s], ph, kTimeoutCycles, abort_flag) ||
-          !ptx::mbar_wait(&afull[s], ph, kTimeoutCycles, abort_flag)) {
+          !ptx::mbar_wait(&afull[a], pa, kTimeoutCycles, abort_flag)) {
         ok = false;
         break;
       }
@@ -182,9 +189,10 @@ tc_decode_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks) {
         const uint64_t bd = ptx::sw128_desc(x_addr + ks * 32, 16, 1024);
-        umma_bf16_ts(tmem, tmem + 32 + 32 * s + 8 * ks, bd, idesc, (i | ks) != 0 ? 1u : 0u);
+        umma_bf16_ts(tmem, tmem + 32 + 32 * a + 8 * ks, bd, idesc, (i | ks) != 0 ? 1u : 0u);
       }
-      ptx::umma_commit(&empty[s]);
+      ptx::umma_commit(&empty[s]);   // the stage may be refilled
+      ptx::umma_commit(&aempty[a]);  // the slot may be rewritten
     }
     for (int tt = 0; tt < k2 && ok; ++tt) {
       if (!ptx::mbar_wait(ext_full, tt & 1, kTimeoutCycles, abort_flag)) break;
@@ -225,16 +233,15 @@ tc_decode_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
     };
     RawScale r0 = load_scale(grp), r1 = load_scale(grp + 2), r2 = load_scale(grp + 4);
     for (int i = grp; i < kn; i += 2) {
-      const int s = i % kStages;
-      const uint32_t ph = (i / kStages) & 1;
+      const int s = i % kStages, a = i % kSlots;
+      const uint32_t ph = (i / kStages) & 1, pa = (i / kSlots) & 1;
       const float sc = !r0.in ? 0.0f
                        : (p.w.dq_shift < 0 ? r0.f : __fadd_rn(__fmul_rn(r0.q, r0.f), mu));
       r0 = r1;
       r1 = r2;
       r2 = load_scale(i + 6);
-      // the stage's codes have landed (and its TMEM slot is free: the producer
-      // refilled the stage only after the MMAs of its previous use completed)
-      // warp-uniform: the TMEM store below is a warp-wide instruction
+      // the stage's codes have landed; warp-uniform: the TMEM store below is a
+      // warp-wide instruction
       if (!__all_sync(0xffffffffu, ptx::mbar_wait(&full[s], ph, kTimeoutCycles, abort_flag))) break;
       const uint8_t* codes = smem + s * kStageBytes + kXBytes + row * 32;
       const uint4 c0 = *reinterpret_cast<const uint4*>(codes);
@@ -253,34 +260,47 @@ tc_decode_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
         v[4 * j + 2] = e.z;
         v[4 * j + 3] = e.w;
       }
-      tmem_st_x32(tmem + (static_cast<uint32_t>(32 * quarter) << 16) + 32 + 32 * s, v);
+      // the slot is free once the MMAs of its previous k-tile have completed
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait(&aempty[a], pa ^ 1, kTimeoutCycles, abort_flag)))
+        break;
+      ptx::tc_fence_after();
+      tmem_st_x32(tmem + (static_cast<uint32_t>(32 * quarter) << 16) + 32 + 32 * a, v);
       tmem_st_wait();
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&afull[s]);
+      if (lane == 0) ptx::mbar_arrive(&afull[a]);
     }
     if (grp == 0) {
       // ---------------------------------------------------------- epilogue
       bool ok = ptx::mbar_wait(accum, 0, kTimeoutCycles, abort_flag);
       ok = __all_sync(0xffffffffu, ok && !*abort_flag);
-      if (ok) {
+      if (p.cluster > 1) {
+        // this split's tile into shared memory, summed over the cluster below
+        uint32_t r[16];
+        if (ok) {
+          ptx::tc_fence_after();
+          ptx::tmem_ld_x16(tmem + (static_cast<uint32_t>(32 * quarter) << 16), r);
+          ptx::tmem_ld_wait();
+        }
+#pragma unroll
+        for (int m = 0; m < 16; ++m)
+          if (m < p.m) red[m * 128 + row] = ok ? __uint_as_float(r[m]) : 0.0f;
+      } else if (ok) {
         ptx::tc_fence_after();
         uint32_t r[16];
         ptx::tmem_ld_x16(tmem + (static_cast<uint32_t>(32 * quarter) << 16), r);
         ptx::tmem_ld_wait();
         const int64_t n = wrow;
         if (n < p.n) {
-          for (int m = 0; m < p.m; ++m) {
-            const int64_t idx = static_cast<int64_t>(blockIdx.y) * p.split_stride +
-                                static_cast<int64_t>(m) * p.n + n;
+#pragma unroll
+          for (int m = 0; m < 16; ++m) {
+            if (m >= p.m) break;
+            const int64_t idx = static_cast<int64_t>(m) * p.n + n;
             if (idx >= p.out_elems) {
               report(p.st, QLORA_ERR_SHAPE, 222u);
               break;
             }
-            if (p.out_bf16)
-              static_cast<__nv_bfloat16*>(p.out)[idx] = __float2bfloat16_rn(__uint_as_float(r[m]));
-            else
-              static_cast<float*>(p.out)[idx] = __uint_as_float(r[m]);
+            p.out[idx] = __float2bfloat16_rn(__uint_as_float(r[m]));
           }
         }
       }
@@ -291,6 +311,33 @@ tc_decode_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
   if (warp == 1) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, kTmemCols);
+  }
+  if (p.cluster > 1) {
+    // the splits of this row tile summed in split order; CTA q of the cluster
+    // writes the tokens m with m % cluster == q
+    ptx::cluster_sync();
+    if (warp >= 2 && warp < 6) {
+      const int row = 32 * (warp & 3) + lane;
+      const int64_t n = static_cast<int64_t>(n0) + row;
+      const int q0 = static_cast<int>(ptx::cluster_ctarank());
+      if (n < p.n) {
+        for (int m = q0; m < p.m; m += p.cluster) {
+          float x[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            x[q] = (q < p.cluster)
+                       ? ptx::ld_cluster_f32(ptx::cluster_addr(&red[m * 128 + row], static_cast<uint32_t>(q)))
+                       : 0.0f;
+          float v = 0.0f;
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            if (q < p.cluster) v += x[q];
+          const int64_t idx = static_cast<int64_t>(m) * p.n + n;
+          if (idx < p.out_elems) p.out[idx] = __float2bfloat16_rn(v);
+        }
+      }
+    }
+    ptx::cluster_sync();  // every CTA keeps its tile until the others have read it
   }
   if (threadIdx.x == 0 && *abort_flag) report(p.st, QLORA_ERR_DEVICE_TIMEOUT, 120u);
 }
@@ -303,7 +350,7 @@ int tc_decode_splits(int64_t M, int64_t N, int64_t K) {
   const int64_t kt = K / 64;
   // two CTAs per SM (TMEM), one wave, at least 8 k-tiles per split
   int64_t s = (2 * 148) / row_tiles;
-  const int64_t max_s = kt / 8 > 0 ? kt / 8 : 1;
+  const int64_t max_s = kt / 8 > 0 ? (kt / 8 < 8 ? kt / 8 : 8) : 1;  // a cluster holds the splits
   if (s > max_s) s = max_s;
   if (s < 1) s = 1;
   const int64_t per = ceil_div(kt, s);
@@ -332,10 +379,9 @@ qlora_status tc_decode_forward(const QView& w, const LevelTable& t, const void* 
   p.w = w;
   p.kblocks = static_cast<int32_t>(K / 64);
   p.nblocks = (N * K / 64) >> w.bs_shift;
-  p.out = out;
-  p.out_bf16 = splits == 1 ? 1 : 0;
-  p.split_stride = M * N;
-  p.out_elems = static_cast<int64_t>(splits) * M * N;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.out_elems = M * N;
+  p.cluster = splits;
   p.st = st;
   static bool configured = false;
   if (!configured) {
@@ -344,11 +390,23 @@ qlora_status tc_decode_forward(const QView& w, const LevelTable& t, const void* 
       return QLORA_ERR_CUDA;
     configured = true;
   }
-  const dim3 grid(static_cast<unsigned>(ceil_div(N, 128)), static_cast<unsigned>(splits));
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(ceil_div(N, 128)), static_cast<unsigned>(splits), 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = static_cast<unsigned>(splits);
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = splits > 1 ? 1 : 0;
   count_launch();
   timing_mark(QLORA_KERNEL_FUSED_FWD, s, true);
-  tc_decode_fwd_kernel<<<grid, kThreads, kSmemBytes, s>>>(mx, mc, mb2, mu2, p, t);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, tc_decode_fwd_kernel, mx, mc, mb2, mu2, p, t);
   timing_mark(QLORA_KERNEL_FUSED_FWD, s, false);
+  if (e != cudaSuccess) return QLORA_ERR_CUDA;
   return after_launch("tc_decode(fwd)", s);
 }
 

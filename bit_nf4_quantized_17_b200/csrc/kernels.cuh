@@ -70,20 +70,22 @@ qlora_status tc2_fused_dgrad(const QView& w, const LevelTable& t, const void* dY
                              const void* sV, const void* A, int32_t r, void* dX,
                              DeviceStatus* st, cudaStream_t s);
 // Forward for M <= 16 tokens with the dequantised W in TMEM as the MMA's A
-// operand (gemm_tc_decode.cu): Y^T = W X^T + B (sU)^T; with splits > 1 `out`
-// receives fp32 partials out[z] of M x N, summed by splitk_reduce.
+// operand (gemm_tc_decode.cu): Y^T = W X^T + B (sU)^T into `out` (M x N bf16);
+// with splits > 1 the CTAs of a row tile form a cluster and sum their
+// contraction splits in shared memory, in split order.
 int tc_decode_splits(int64_t M, int64_t N, int64_t K);
 qlora_status tc_decode_forward(const QView& w, const LevelTable& t, const void* X, int64_t M,
                                const void* sU, const void* B, int32_t r, void* out, int splits,
                                DeviceStatus* st, cudaStream_t s);
 // Dequant GEMV for the dX product of one or two tokens on the CUDA cores
-// (gemv_small.cu): partials part[c][m][k] of dY W + s V A (V fp32), summed
-// over gemv_dgrad_chunks(M, K) chunks.
+// (gemv_small.cu): partials part[c][m][k] of dY W + s V A (V fp32), one per
+// cluster of row chunks; *parts (at most gemv_dgrad_parts(M, K), the
+// workspace bound) is the number written, to be summed by splitk_reduce.
 bool gemv_eligible(int64_t M, int64_t K, int32_t r);
-int gemv_dgrad_chunks(int64_t M, int64_t K);
+int gemv_dgrad_parts(int64_t M, int64_t K);
 qlora_status gemv_dgrad(const QView& w, const LevelTable& t, const void* dY, int64_t M,
                         const float* V, const void* A, int32_t r, float s, float* part,
-                        cudaStream_t st);
+                        int* parts, cudaStream_t st);
 // part[z] (m_rows x n_cols fp32) = A . B^T over split z of the contraction; B has
 // b_rows rows, read as n_cols (rows past b_rows are zero).
 qlora_status tc_lora_gemm(const void* A, bool a_mn, int64_t m_rows, int64_t kdim, int64_t ld_a,
@@ -118,6 +120,27 @@ qlora_status splitk_reduce(const ReduceArgs& a, cudaStream_t s);
 qlora_status transpose_to_bf16(const void* in, bool in_f32, int64_t rows, int cols, int64_t ld_in,
                                void* out, int64_t ld_out, int lo_rows, cudaStream_t s);
 
+// lora_decode.cu: U = X A^T and V = dY B for M <= 16 tokens in one launch each
+// (cluster-reduced, deterministic).  Outputs for token m < M, rank column j:
+//   o1[m ld1 + j] = a1 v (j < r),  o2[m ld2 + j] = hi(a2 v), o2[m ld2 + j + o2_lo] =
+//   lo(a2 v) (j < r; zeros for r <= j < o2_lo), v masked to 0 when seg[m] != j / seg_cols.
+struct RankOut {
+  int32_t r;
+  float* o1;
+  int64_t ld1;
+  float a1;
+  __nv_bfloat16* o2;
+  int64_t ld2;
+  float a2;
+  int32_t o2_lo;
+  const int32_t* seg;
+  int32_t seg_cols;
+};
+qlora_status rank_down(const void* X, const void* A, int M, int64_t K, int32_t span,
+                       const RankOut& o, cudaStream_t s);
+qlora_status rank_v(const void* dY, const void* B, int M, int64_t N, int32_t span,
+                    const RankOut& o, cudaStream_t s);
+
 // dropout.cu: X_drop = X (.) D (mask bit (k % 8) of byte m K / 8 + k / 8 keeps
 // X[m][k]; K a multiple of 8), and dX[m][k] += D[m][k] scale (V A)[m][k] in place.
 qlora_status dropout_apply(const void* X, const uint8_t* mask, int64_t M, int64_t K, void* X_drop,
@@ -125,15 +148,8 @@ qlora_status dropout_apply(const void* X, const uint8_t* mask, int64_t M, int64_
 qlora_status dropout_dx(void* dX, const float* V, int64_t ldv, const void* A, const uint8_t* mask,
                         int64_t M, int64_t K, int32_t r, float scale, cudaStream_t s);
 
-// lora_small.cu: LoRA-side kernels for M <= 16 tokens (CUDA cores).
+// lora_small.cu: dA and dB for M <= 16 tokens (CUDA cores); r a multiple of 8.
 constexpr int kSmallM = 16;
-int small_chunks(int64_t len);  // partial count of the two reductions below
-// part[z][m][j] (z over 256-wide chunks of d_in, row stride lora_rows(r)) of X A^T
-qlora_status small_down_partial(const void* X, const void* A, int M, int64_t K, int r,
-                                float* part, cudaStream_t s);
-// part[z][m][j] (z over 256-row chunks of d_out) of dY B
-qlora_status small_v_partial(const void* dY, const void* B, int M, int64_t N, int r, float* part,
-                             cudaStream_t s);
 qlora_status small_grad_b(const void* dY, const float* U, int M, int64_t N, int r, float sc,
                           bool accumulate, float* dB, cudaStream_t s);
 qlora_status small_grad_a(const float* V, const void* X, int M, int64_t K, int r, float sc,

@@ -84,30 +84,25 @@ TcLayout tc_layout(int64_t M, int64_t N, int64_t K, int32_t r) {
 }
 
 // Workspace of the decode-sized path (M <= 16, tensor-core conditions):
-//   forward   sU [hi | lo] | U-partials | fused partials
-//   backward  sV [hi | lo] | V (fp32) | U (fp32, when recomputed) | partials | fused partials
+//   forward   sU [hi | lo]
+//   backward  sV [hi | lo] | V (fp32) | U (fp32, when recomputed) | fused partials
 struct SmallLayout {
-  size_t su, part_f, fused_f, fwd_end, sv, v, u, part_b, fused_b, bwd_end;
+  size_t su, fwd_end, sv, v, u, fused_b, bwd_end;
 };
 
 SmallLayout small_layout(int64_t M, int64_t N, int64_t K, int32_t r) {
-  const int64_t r16 = lora_rows(r), span = lora_span(r);
+  const int64_t span = lora_span(r);
   SmallLayout L{};
   L.su = kStatusBytes;
-  L.part_f = L.su + align256(2 * M * 2 * span);
-  L.fused_f = L.part_f + align256(sizeof(float) * small_chunks(K) * M * r16);
-  const FusedShape ff = fused_shape(M, N, K / 64);
-  const int fsplits = std::max(ff.splits, tc_decode_splits(M, N, K));
-  L.fwd_end = L.fused_f + (fsplits > 1 ? align256(sizeof(float) * fsplits * M * N) : 0);
+  L.fwd_end = L.su + align256(2 * M * 2 * span);
   L.sv = kStatusBytes;
   L.v = L.sv + align256(2 * M * 2 * span);
   L.u = L.v + align256(sizeof(float) * M * r);
-  L.part_b = L.u + align256(sizeof(float) * M * r);
-  L.fused_b = L.part_b + align256(sizeof(float) * std::max(small_chunks(K), small_chunks(N)) * M * r16);
+  L.fused_b = L.u + align256(sizeof(float) * M * r);
   const FusedShape fb = fused_shape(M, K, ceil_div(N, 64));
   const size_t fused_parts = fb.splits > 1 ? sizeof(float) * fb.splits * M * K : 0;
   const size_t gemv_parts =
-      gemv_eligible(M, K, r) ? sizeof(float) * gemv_dgrad_chunks(M, K) * M * K : 0;
+      gemv_eligible(M, K, r) ? sizeof(float) * gemv_dgrad_parts(M, K) * M * K : 0;
   L.bwd_end = L.fused_b + align256(std::max(fused_parts, gemv_parts));
   return L;
 }
@@ -202,32 +197,15 @@ qlora_status linear_forward(const qlora_nf4& W, const LevelTable& t, const void*
   }
   if (use_tc(M, N, K, r) && use_small(M)) {
     const SmallLayout L = small_layout(M, N, K, r);
-    const int32_t r16 = lora_rows(r), span = lora_span(r);
+    const int32_t span = lora_span(r);
     char* su = ws + L.su;
-    float* part = reinterpret_cast<float*>(ws + L.part_f);
-    QLORA_TRY(small_down_partial(xl, A, static_cast<int>(M), K, r, part, s));
-    ReduceArgs ra = reduce_args(part, small_chunks(K), M, r, r16);
-    ra.seg = seg;  // U / V: each token keeps only its adapter's columns
-    ra.seg_cols = r_adapter;
-    ra.o1 = U_save;
-    ra.ld1 = r;
-    ra.a1 = o.keep;
-    ra.o2 = su;
-    ra.ld2 = 2 * span;
-    ra.a2 = sc * o.keep;
-    ra.o2_lo = span;
-    ra.o2_pad = 1;  // the padding columns meet zero B columns in the MMA: written as zeros
-    QLORA_TRY(splitk_reduce(ra, s));
-    // Y = X W^T + sU B^T with W in TMEM as the MMA's A operand
-    const int splits = tc_decode_splits(M, N, K);
-    if (splits == 1) return tc_decode_forward(w, t, X, M, su, B, r, Y, 1, st, s);
-    float* fpart = reinterpret_cast<float*>(ws + L.fused_f);
-    QLORA_TRY(tc_decode_forward(w, t, X, M, su, B, r, fpart, splits, st, s));
-    ReduceArgs ry = reduce_args(fpart, splits, M, static_cast<int>(N), static_cast<int>(N));
-    ry.o2 = Y;
-    ry.ld2 = N;
-    ry.a2 = 1.0f;
-    return splitk_reduce(ry, s);
+    // U = X A^T -> U_save (fp32) and sU = s U as bf16 hi + lo, one launch
+    const RankOut ro{r, U_save, r, o.keep, reinterpret_cast<__nv_bfloat16*>(su), 2 * span,
+                     sc * o.keep, span, seg, r_adapter};
+    QLORA_TRY(rank_down(xl, A, static_cast<int>(M), K, span, ro, s));
+    // Y = X W^T + sU B^T with W in TMEM as the MMA's A operand; the splits of
+    // the contraction are summed inside their cluster
+    return tc_decode_forward(w, t, X, M, su, B, r, Y, tc_decode_splits(M, N, K), st, s);
   }
   if (use_tc(M, N, K, r)) {
     const TcLayout L = tc_layout(M, N, K, r);
@@ -296,47 +274,27 @@ qlora_status linear_backward(const qlora_nf4& W, const LevelTable& t, const void
   auto* st = reinterpret_cast<DeviceStatus*>(ws);
   if (use_tc(M, N, K, r) && use_small(M)) {
     const SmallLayout L = small_layout(M, N, K, r);
-    const int32_t r16 = lora_rows(r), span = lora_span(r);
+    const int32_t span = lora_span(r);
     const int m = static_cast<int>(M);
     char* sv = ws + L.sv;
     float* v = reinterpret_cast<float*>(ws + L.v);
-    float* part = reinterpret_cast<float*>(ws + L.part_b);
     const bool gemv = gemv_eligible(M, K, r);
     // V = dY B -> V (fp32) and, for the tensor-core kernel, sV = s V as [hi | lo]
-    QLORA_TRY(small_v_partial(dY, B, m, N, r, part, s));
-    {
-      ReduceArgs ra = reduce_args(part, small_chunks(N), M, r, r16);
-      ra.seg = seg;  // U / V: each token keeps only its adapter's columns
-      ra.seg_cols = r_adapter;
-      ra.o1 = v;
-      ra.ld1 = r;
-      ra.a1 = 1.0f;
-      if (!gemv) {
-        ra.o2 = sv;
-        ra.ld2 = 2 * span;
-        ra.a2 = sc_dx;
-        ra.o2_lo = span;
-        ra.o2_pad = 1;
-      }
-      QLORA_TRY(splitk_reduce(ra, s));
-    }
+    const RankOut rv{r, v, r, 1.0f, gemv ? nullptr : reinterpret_cast<__nv_bfloat16*>(sv),
+                     2 * span, sc_dx, span, seg, r_adapter};
+    QLORA_TRY(rank_v(dY, B, m, N, span, rv, s));
     if (!U) {
       float* u = reinterpret_cast<float*>(ws + L.u);
-      QLORA_TRY(small_down_partial(xl, A, m, K, r, part, s));
-      ReduceArgs ra = reduce_args(part, small_chunks(K), M, r, r16);
-      ra.seg = seg;  // U / V: each token keeps only its adapter's columns
-      ra.seg_cols = r_adapter;
-      ra.o1 = u;
-      ra.ld1 = r;
-      ra.a1 = o.keep;
-      QLORA_TRY(splitk_reduce(ra, s));
+      const RankOut ru{r, u, r, o.keep, nullptr, 0, 0.0f, 0, seg, r_adapter};
+      QLORA_TRY(rank_down(xl, A, m, K, span, ru, s));
       U = u;
     }
     if (dX && gemv) {
       // dX = dY W + s V A: CTA partials of the dequant GEMV, summed in order
       float* fpart = reinterpret_cast<float*>(ws + L.fused_b);
-      QLORA_TRY(gemv_dgrad(w, t, dY, M, v, A, r, sc_dx, fpart, s));
-      ReduceArgs rx = reduce_args(fpart, gemv_dgrad_chunks(M, K), M, static_cast<int>(K),
+      int parts = 0;
+      QLORA_TRY(gemv_dgrad(w, t, dY, M, v, A, r, sc_dx, fpart, &parts, s));
+      ReduceArgs rx = reduce_args(fpart, parts, M, static_cast<int>(K),
                                   static_cast<int>(K));
       rx.o2 = dX;
       rx.ld2 = K;

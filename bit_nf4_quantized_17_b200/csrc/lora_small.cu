@@ -1,15 +1,11 @@
-// LoRA-side contractions for decode-sized batches (M <= 16 tokens).
+// LoRA gradients for decode-sized batches (M <= 16 tokens).
 //
-// With so few tokens the rank-r branch ("LoRA 与 QLoRA：把大模型微调拆成可负担
-// 的工程", 2: h = W x + (alpha/r) B A x) is a handful of short reductions and
-// rank-M outer products, bound by reading A and B and writing dA and dB:
+// With so few tokens dA and dB of the rank-r branch ("LoRA 与 QLoRA：把大模型
+// 微调拆成可负担的工程", 2: h = W x + (alpha/r) B A x) are rank-M outer
+// products, bound by writing dA and dB:
 //
-//   down_partial  part[z][m][j] = sum_{k in chunk z} X[m][k] A[j][k]    (U = X A^T)
-//   v_partial     part[z][m][j] = sum_{n in chunk z} dY[m][n] B[n][j]   (V = dY B)
 //   grad_b        dB[n][j] = s sum_m dY[m][n] U[m][j]   (+ dB)
 //   grad_a        dA[j][k] = s sum_m V[m][j] X[m][k]    (+ dA)
-//
-// The partials are summed in a fixed order by splitk_reduce (deterministic).
 #include "internal.cuh"
 #include "kernels.cuh"
 
@@ -17,118 +13,84 @@ namespace qlora {
 namespace {
 
 constexpr int kMaxM = 16;
-constexpr int kChunk = 64;
 
-// One CTA per chunk of 64 k; warp w handles ranks j = w, w + 8, ...; lanes
-// stride over k; X chunk staged in shared memory.
-__global__ void __launch_bounds__(256)
-down_partial_kernel(const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict__ A,
-                    int M, int64_t K, int r, int r16, float* __restrict__ part) {
-  __shared__ float xs[kMaxM][kChunk];
-  const int64_t k0 = static_cast<int64_t>(blockIdx.x) * kChunk;
-  const int kc = static_cast<int>((K - k0) < kChunk ? (K - k0) : kChunk);
-  for (int e = threadIdx.x; e < M * kChunk; e += 256) {
-    const int m = e / kChunk, k = e % kChunk;
-    xs[m][k] = (k < kc) ? __bfloat162float(X[m * K + k0 + k]) : 0.0f;
-  }
-  __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float* out = part + static_cast<int64_t>(blockIdx.x) * M * r16;
-  for (int j = warp; j < r; j += 8) {
-    float acc[kMaxM];
-#pragma unroll
-    for (int m = 0; m < kMaxM; ++m) acc[m] = 0.0f;
-    const __nv_bfloat16* arow = A + j * K + k0;
-    for (int k = lane; k < kc; k += 32) {
-      const float a = __bfloat162float(arow[k]);
-#pragma unroll
-      for (int m = 0; m < kMaxM; ++m)
-        if (m < M) acc[m] = fmaf(xs[m][k], a, acc[m]);
-    }
-#pragma unroll
-    for (int m = 0; m < kMaxM; ++m) {
-      if (m >= M) break;
-      float v = acc[m];
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-      if (lane == 0) out[m * r16 + j] = v;
-    }
-  }
-}
-
-// One CTA per chunk of 64 rows n (dY chunk staged in shared memory); thread t
-// covers rank j = t % r and row lane t / r; the row lanes are summed in
-// shared memory.
-__global__ void __launch_bounds__(256)
-v_partial_kernel(const __nv_bfloat16* __restrict__ dY, const __nv_bfloat16* __restrict__ B,
-                 int M, int64_t N, int r, int r16, float* __restrict__ part) {
-  __shared__ float ys[kMaxM][kChunk];
-  __shared__ float red[256][kMaxM + 1];
-  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kChunk;
-  const int nc = static_cast<int>((N - n0) < kChunk ? (N - n0) : kChunk);
-  for (int e = threadIdx.x; e < M * kChunk; e += 256) {
-    const int m = e / kChunk, n = e % kChunk;
-    ys[m][n] = (n < nc) ? __bfloat162float(dY[m * N + n0 + n]) : 0.0f;
-  }
-  __syncthreads();
-  const int lanes = 256 / r;
-  const int j = threadIdx.x % r, nl = threadIdx.x / r;
-  float acc[kMaxM];
-#pragma unroll
-  for (int m = 0; m < kMaxM; ++m) acc[m] = 0.0f;
-  if (nl < lanes) {
-    for (int n = nl; n < nc; n += lanes) {
-      const float b = __bfloat162float(B[(n0 + n) * r + j]);
-#pragma unroll
-      for (int m = 0; m < kMaxM; ++m)
-        if (m < M) acc[m] = fmaf(ys[m][n], b, acc[m]);
-    }
-  }
-#pragma unroll
-  for (int m = 0; m < kMaxM; ++m) red[threadIdx.x][m] = acc[m];
-  __syncthreads();
-  float* out = part + static_cast<int64_t>(blockIdx.x) * M * r16;
-  for (int e = threadIdx.x; e < M * r; e += 256) {
-    const int m = e / r, jj = e % r;
-    float v = 0.0f;
-    for (int l = 0; l < lanes; ++l) v += red[l * r + jj][m];
-    out[m * r16 + jj] = v;
-  }
-}
-
-// dB[n][j] = s sum_m dY[m][n] U[m][j]  (+ dB)
+// dB[n][j..j+3] = s sum_m dY[m][n] U[m][j..j+3]  (+ dB); one thread per 4 ranks of a row
+template <int MM>
 __global__ void __launch_bounds__(256)
 grad_b_kernel(const __nv_bfloat16* __restrict__ dY, const float* __restrict__ U, int M, int64_t N,
               int r, float s, int accumulate, float* __restrict__ dB) {
-  __shared__ float us[kMaxM * 256];
+  __shared__ __align__(16) float us[kMaxM * 256];
   for (int e = threadIdx.x; e < M * r; e += 256) us[e] = U[e];
   __syncthreads();
-  const int64_t total = N * r;
+  const int q4 = r / 4;
+  const int64_t total = N * q4;
   for (int64_t e = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; e < total;
        e += static_cast<int64_t>(gridDim.x) * 256) {
-    const int64_t n = e / r;
-    const int j = static_cast<int>(e - n * r);
-    float v = 0.0f;
-    for (int m = 0; m < M; ++m) v = fmaf(__bfloat162float(dY[m * N + n]), us[m * r + j], v);
-    dB[e] = accumulate ? dB[e] + s * v : s * v;
+    const int64_t n = e / q4;
+    const int j = 4 * static_cast<int>(e - n * q4);
+    float dy[MM];
+#pragma unroll
+    for (int m = 0; m < MM; ++m) dy[m] = (m < M) ? __bfloat162float(dY[m * N + n]) : 0.0f;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int m = 0; m < MM; ++m) {
+      if (m >= M) break;
+      const float4 u = *reinterpret_cast<const float4*>(&us[m * r + j]);
+      v.x = fmaf(dy[m], u.x, v.x);
+      v.y = fmaf(dy[m], u.y, v.y);
+      v.z = fmaf(dy[m], u.z, v.z);
+      v.w = fmaf(dy[m], u.w, v.w);
+    }
+    float4* dst = reinterpret_cast<float4*>(dB + n * r + j);
+    float4 o = make_float4(s * v.x, s * v.y, s * v.z, s * v.w);
+    if (accumulate) {
+      const float4 d = *dst;
+      o = make_float4(d.x + o.x, d.y + o.y, d.z + o.z, d.w + o.w);
+    }
+    *dst = o;
   }
 }
 
-// dA[j][k] = s sum_m V[m][j] X[m][k]  (+ dA)
+// dA[j][k..k+7] = s sum_m V[m][j] X[m][k..k+7]  (+ dA); one thread per 8 columns of a rank
+template <int MM>
 __global__ void __launch_bounds__(256)
 grad_a_kernel(const float* __restrict__ V, const __nv_bfloat16* __restrict__ X, int M, int64_t K,
               int r, float s, int accumulate, float* __restrict__ dA) {
   __shared__ float vs[kMaxM * 256];
   for (int e = threadIdx.x; e < M * r; e += 256) vs[e] = V[e];
   __syncthreads();
-  const int64_t total = static_cast<int64_t>(r) * K;
+  const int64_t k8 = K / 8;
+  const int64_t total = static_cast<int64_t>(r) * k8;
   for (int64_t e = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; e < total;
        e += static_cast<int64_t>(gridDim.x) * 256) {
-    const int j = static_cast<int>(e / K);
-    const int64_t k = e - static_cast<int64_t>(j) * K;
-    float v = 0.0f;
-    for (int m = 0; m < M; ++m) v = fmaf(vs[m * r + j], __bfloat162float(X[m * K + k]), v);
-    dA[e] = accumulate ? dA[e] + s * v : s * v;
+    const int j = static_cast<int>(e / k8);
+    const int64_t k = 8 * (e - static_cast<int64_t>(j) * k8);
+    uint4 xr[MM];
+#pragma unroll
+    for (int m = 0; m < MM; ++m)
+      xr[m] = (m < M) ? *reinterpret_cast<const uint4*>(X + m * K + k) : make_uint4(0u, 0u, 0u, 0u);
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int m = 0; m < MM; ++m) {
+      if (m >= M) break;
+      const float v = vs[m * r + j];
+      const uint32_t w[4] = {xr[m].x, xr[m].y, xr[m].z, xr[m].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        acc[2 * q] = fmaf(v, __uint_as_float(w[q] << 16), acc[2 * q]);
+        acc[2 * q + 1] = fmaf(v, __uint_as_float(w[q] & 0xffff0000u), acc[2 * q + 1]);
+      }
+    }
+    float4* dst = reinterpret_cast<float4*>(dA + static_cast<int64_t>(j) * K + k);
+    float4 o0 = make_float4(s * acc[0], s * acc[1], s * acc[2], s * acc[3]);
+    float4 o1 = make_float4(s * acc[4], s * acc[5], s * acc[6], s * acc[7]);
+    if (accumulate) {
+      const float4 d0 = dst[0], d1 = dst[1];
+      o0 = make_float4(d0.x + o0.x, d0.y + o0.y, d0.z + o0.z, d0.w + o0.w);
+      o1 = make_float4(d1.x + o1.x, d1.y + o1.y, d1.z + o1.z, d1.w + o1.w);
+    }
+    dst[0] = o0;
+    dst[1] = o1;
   }
 }
 
@@ -139,43 +101,29 @@ int grid_cap(int64_t items) {
 
 }  // namespace
 
-int small_chunks(int64_t len) { return static_cast<int>(ceil_div(len, kChunk)); }
-
-qlora_status small_down_partial(const void* X, const void* A, int M, int64_t K, int r,
-                                float* part, cudaStream_t s) {
-  if (M > kMaxM) return QLORA_ERR_UNSUPPORTED;
-  count_launch();
-  down_partial_kernel<<<small_chunks(K), 256, 0, s>>>(
-      static_cast<const __nv_bfloat16*>(X), static_cast<const __nv_bfloat16*>(A), M, K, r,
-      lora_rows(r), part);
-  return after_launch("small_down_partial", s);
-}
-
-qlora_status small_v_partial(const void* dY, const void* B, int M, int64_t N, int r, float* part,
-                             cudaStream_t s) {
-  if (M > kMaxM) return QLORA_ERR_UNSUPPORTED;
-  count_launch();
-  v_partial_kernel<<<small_chunks(N), 256, 0, s>>>(static_cast<const __nv_bfloat16*>(dY),
-                                                   static_cast<const __nv_bfloat16*>(B), M, N, r,
-                                                   lora_rows(r), part);
-  return after_launch("small_v_partial", s);
-}
-
 qlora_status small_grad_b(const void* dY, const float* U, int M, int64_t N, int r, float sc,
                           bool accumulate, float* dB, cudaStream_t s) {
-  if (M > kMaxM) return QLORA_ERR_UNSUPPORTED;
+  if (M > kMaxM || r % 8 != 0) return QLORA_ERR_UNSUPPORTED;
+  const int g = grid_cap(N * (r / 4));
+  const auto* y = static_cast<const __nv_bfloat16*>(dY);
+  const int acc = accumulate ? 1 : 0;
   count_launch();
-  grad_b_kernel<<<grid_cap(N * r), 256, 0, s>>>(static_cast<const __nv_bfloat16*>(dY), U, M, N, r,
-                                                sc, accumulate ? 1 : 0, dB);
+  if (M == 1) grad_b_kernel<1><<<g, 256, 0, s>>>(y, U, M, N, r, sc, acc, dB);
+  else if (M <= 4) grad_b_kernel<4><<<g, 256, 0, s>>>(y, U, M, N, r, sc, acc, dB);
+  else grad_b_kernel<16><<<g, 256, 0, s>>>(y, U, M, N, r, sc, acc, dB);
   return after_launch("small_grad_b", s);
 }
 
 qlora_status small_grad_a(const float* V, const void* X, int M, int64_t K, int r, float sc,
                           bool accumulate, float* dA, cudaStream_t s) {
-  if (M > kMaxM) return QLORA_ERR_UNSUPPORTED;
+  if (M > kMaxM || K % 8 != 0) return QLORA_ERR_UNSUPPORTED;
+  const int g = grid_cap(r * (K / 8));
+  const auto* x = static_cast<const __nv_bfloat16*>(X);
+  const int acc = accumulate ? 1 : 0;
   count_launch();
-  grad_a_kernel<<<grid_cap(K * r), 256, 0, s>>>(V, static_cast<const __nv_bfloat16*>(X), M, K, r,
-                                                sc, accumulate ? 1 : 0, dA);
+  if (M == 1) grad_a_kernel<1><<<g, 256, 0, s>>>(V, x, M, K, r, sc, acc, dA);
+  else if (M <= 4) grad_a_kernel<4><<<g, 256, 0, s>>>(V, x, M, K, r, sc, acc, dA);
+  else grad_a_kernel<16><<<g, 256, 0, s>>>(V, x, M, K, r, sc, acc, dA);
   return after_launch("small_grad_a", s);
 }
 

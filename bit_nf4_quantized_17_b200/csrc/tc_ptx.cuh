@@ -145,6 +145,14 @@ __device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
   return a;
 }
+// Load of an fp32 from another CTA's shared memory (its shared::cluster
+// address).  Not volatile and without a memory clobber, so that independent
+// loads overlap: callers place it between cluster barriers, which order it.
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
+  float v;
+  asm("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  return v;
+}
 // Arrive on an mbarrier given by its shared::cluster address (default
 // semantics).  Used after fence.proxy.async by threads whose shared-memory
 // writes the pair MMA reads: the proxy fence orders the writes for the
