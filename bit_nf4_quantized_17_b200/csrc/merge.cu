@@ -28,7 +28,10 @@ merge_kernel(QView w, LevelTable tab, const __nv_bfloat16* __restrict__ A,
   const int64_t n0 = static_cast<int64_t>(blockIdx.y) * kRows;
   const int64_t k0 = static_cast<int64_t>(blockIdx.x) * kCols;
   const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;  // rows 4 ty .., columns 8 tx ..
-  if (threadIdx.x < 16) lv[threadIdx.x] = tab.level[threadIdx.x];
+  if (threadIdx.x == 0) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) lv[j] = tab.level[j];  // constant indices: no local copy
+  }
   float acc[4][8];
 #pragma unroll
   for (int i = 0; i < 4; ++i)
