@@ -404,24 +404,50 @@ def run_ours(args):
     torch.cuda.synchronize()
     barrier(world)
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    # events recorded inside a CUDA graph must be external to be recorded when it runs
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)]
+           for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    launches0 = Q.qlora_launch_count()
     # per-kernel CUDA events, recorded by the library on the launching stream
     # around the two fused kernels (the dominant ones) inside the timed region
     fused_kinds = (Q.QLORA_KERNEL_FUSED_FWD, Q.QLORA_KERNEL_FUSED_DGRAD)
+    use_graph = world == 1 and not args.eager
+    graph = None
+    if use_graph:
+        # the K timed steps captured as one CUDA graph (launched once below):
+        # the same kernels with the host's launch gaps taken out
+        launches0 = Q.qlora_launch_count()
+        Q.qlora_timing_begin(fused_kinds, max_launches=4 * args.steps)
+        graph = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream()
+        cap.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(cap):
+            with torch.cuda.graph(graph, stream=cap):
+                for i in range(args.steps):
+                    run_step(sets[i % N_SETS], shape, Q, ev=evs[i], world=world)
+        torch.cuda.current_stream().wait_stream(cap)
+        launches = Q.qlora_launch_count() - launches0
+        torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         barrier(world)
         torch.cuda.synchronize()
-        Q.qlora_timing_begin(fused_kinds, max_launches=4 * args.steps)
-        start.record()
-        for i in range(args.steps):
-            run_step(sets[i % N_SETS], shape, Q, ev=evs[i], world=world)
-        end.record()
+        if use_graph:
+            start.record()
+            graph.replay()
+            end.record()
+        else:
+            launches0 = Q.qlora_launch_count()
+            Q.qlora_timing_begin(fused_kinds, max_launches=4 * args.steps)
+            start.record()
+            for i in range(args.steps):
+                run_step(sets[i % N_SETS], shape, Q, ev=evs[i], world=world)
+            end.record()
+            launches = Q.qlora_launch_count() - launches0
         torch.cuda.synchronize()
+        # the graph refers to the library's timing events: release it first
+        del graph
         kt = Q.qlora_timing_end()
         barrier(world)
-    launches = Q.qlora_launch_count() - launches0
     # the other kernels in a second pass over the same steps (their events
     # would otherwise add a gap to every launch of the timed region)
     Q.qlora_timing_begin((Q.QLORA_KERNEL_QUANTIZE, Q.QLORA_KERNEL_LORA_GEMM),
@@ -505,7 +531,8 @@ def run_ours(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,.) tensors of the workload's shapes)",
-        "config": workload_config(world),
+        "config": dict(workload_config(world),
+                       launch="one CUDA graph of the timed steps" if use_graph else "eager"),
         "nf4_weight_gbs": round(2 * wb / (t_fwd + t_bwd) / 1e9, 1),
         "fwd_ms": round(t_fwd * 1e3, 4), "bwd_ms": round(t_bwd * 1e3, 4),
         "fwd_tflops": round(fwd_flops(M, N, K, r) / t_fwd / 1e12, 2),
@@ -656,6 +683,8 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--eager", action="store_true",
+                    help="launch the timed steps one call at a time instead of one CUDA graph")
     ap.add_argument("--workload", default=WORKLOAD, choices=[WORKLOAD] + sorted(CONFIGS),
                     help="another workload of the problem (one GPU, our arm only)")
     args = ap.parse_args(argv)

@@ -29,7 +29,31 @@ struct Timing {
 Timing g_timing;
 }  // namespace
 
-void qlora::count_launch(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+void qlora::count_launch(unsigned n) {
+  g_launches.fetch_add(n, std::memory_order_relaxed);
+  // every launch is followed by after_launch, which reads the thread's last
+  // error: clear one left by an unrelated earlier call so that it reports this launch
+  (void)cudaGetLastError();
+}
+
+namespace {
+// Record a timing event.  Inside a stream capture the record must be external
+// to become a graph node that records the event when the graph runs; outside
+// a capture the plain record is used.  A failed record leaves no error behind
+// for the launch checks to report: the launch is not timed, nothing else.
+bool record_timing_event(cudaEvent_t ev, cudaStream_t s) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return false;
+  }
+  const cudaError_t e = (cs == cudaStreamCaptureStatusActive)
+                            ? cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal)
+                            : cudaEventRecord(ev, s);
+  if (e != cudaSuccess) (void)cudaGetLastError();
+  return e == cudaSuccess;
+}
+}  // namespace
 
 void qlora::timing_mark(int kind, cudaStream_t s, bool start) {
   if (!g_timing.on.load(std::memory_order_acquire)) return;
@@ -38,13 +62,13 @@ void qlora::timing_mark(int kind, cudaStream_t s, bool start) {
   const int cap = static_cast<int>(g_timing.kind.size());
   if (start) {
     if (g_timing.used >= cap) return;
-    if (cudaEventRecord(g_timing.ev[2 * g_timing.used], s) == cudaSuccess) {
+    if (record_timing_event(g_timing.ev[2 * g_timing.used], s)) {
       g_timing.kind[g_timing.used] = kind;
       g_timing.open = true;
     }
   } else if (g_timing.open) {
     g_timing.open = false;
-    if (cudaEventRecord(g_timing.ev[2 * g_timing.used + 1], s) == cudaSuccess) ++g_timing.used;
+    if (record_timing_event(g_timing.ev[2 * g_timing.used + 1], s)) ++g_timing.used;
   }
 }
 

@@ -301,7 +301,9 @@ uint64_t qlora_launch_count(void);
  * device time in milliseconds and the launch count of each kind to
  * ms[QLORA_KERNEL_KINDS] and launches[QLORA_KERNEL_KINDS] (either may be
  * NULL), and releases the events.  The events are library-owned host
- * objects; no device memory is allocated.  Launches from several host
+ * objects; no device memory is allocated.  Calls captured into a CUDA graph
+ * while timing is on record their events as graph nodes: qlora_timing_end,
+ * after the graph has run, reads the times of that run.  Launches from several host
  * threads at once are not supported while timing is on.
  * Errors: QLORA_ERR_SHAPE for max_launches outside [1, 65536],
  * QLORA_ERR_UNSUPPORTED for begin while timing is already on or end while it
