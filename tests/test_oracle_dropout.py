@@ -83,3 +83,18 @@ def test_inverted_dropout_is_unbiased():
     ref = x @ a.T
     se = np.sqrt(p / (1 - p) * (x * x) @ (a * a).T / n)   # standard error of each mean
     assert np.all(np.abs(mean - ref) < 5 * se)
+
+
+def test_binding_mask_packing_matches_the_oracle_layout():
+    # the binding's keep-mask helper (torch's generator, any device) packs bit
+    # k % 8 of byte [m][k // 8]; the oracle unpacks it back to the draw
+    import torch
+
+    from bit_nf4_quantized_17_b200 import qlora as Q
+
+    g = torch.Generator().manual_seed(3)
+    m = Q.dropout_keep_mask(4, 64, 0.3, generator=g, device="cpu")
+    g2 = torch.Generator().manual_seed(3)
+    keep = (torch.rand((4, 8, 8), generator=g2) >= 0.3).reshape(4, 64).numpy()
+    assert m.shape == (4, 8) and m.dtype == torch.uint8
+    assert np.array_equal(oracle.unpack_keep_mask(m.numpy(), 64), keep.astype(np.float64))
