@@ -31,7 +31,9 @@
  *   - Argument errors are found on the host and returned before any launch.
  *     Errors found on the device (a non-finite weight, a bounded wait that
  *     gave up) are written to a status word at the start of the workspace;
- *     qlora_check() synchronises the stream and returns it.
+ *     qlora_check() synchronises the stream and returns it.  A workspace must
+ *     be zero-filled before its first use; the library leaves its status word
+ *     zero unless it reports an error (qlora_check clears it again).
  *   - No call exits, aborts or traps.
  */
 #ifndef QLORA_H
