@@ -261,6 +261,17 @@ qlora_status qlora_merge(const qlora_nf4* W, const void* A, const void* B, int32
   return launch_merge(*W, *t, A, B, r, alpha, W_out, static_cast<cudaStream_t>(stream));
 }
 
+qlora_status qlora_merge_dense(const void* W_in, int64_t rows, int64_t cols, const void* A,
+                               const void* B, int32_t r, float alpha, void* W_out, void* stream) {
+  if (!W_in || !A || !B || !W_out) return QLORA_ERR_NULL;
+  if (rows < 1 || cols < 1 || cols % 8 != 0 || r < 1 || r > 256 || rows > (int64_t(1) << 22))
+    return QLORA_ERR_SHAPE;
+  if (!aligned16(W_in) || !aligned16(A) || !aligned16(B) || !aligned16(W_out))
+    return QLORA_ERR_ALIGN;
+  return launch_merge_dense(W_in, rows, cols, A, B, r, alpha, W_out,
+                            static_cast<cudaStream_t>(stream));
+}
+
 qlora_status qlora_linear_workspace(int64_t M, int64_t N, int64_t K, int32_t r, size_t* fwd_bytes,
                                     size_t* bwd_bytes) {
   if (M < 0 || N < 1 || K < 1 || r < 1 || r > 256) return QLORA_ERR_SHAPE;

@@ -68,6 +68,9 @@ qlora_status launch_adamw(float* p, void* p16, const float* g, float* m, float* 
 // merge.cu: W_out = bf16(dequant(W) + (alpha / r) B A)
 qlora_status launch_merge(const qlora_nf4& q, const LevelTable& t, const void* A, const void* B,
                           int32_t r, float alpha, void* out, cudaStream_t s);
+// merge.cu: W_out = bf16(W_in + (alpha / r) B A) for a dense bf16 W_in (may alias W_out)
+qlora_status launch_merge_dense(const void* W_in, int64_t rows, int64_t cols, const void* A,
+                                const void* B, int32_t r, float alpha, void* out, cudaStream_t s);
 
 // Everything a linear-layer kernel needs to read a quantised W.
 struct QView {

@@ -101,6 +101,7 @@ def lib():
                                                    vp, vp, i32, vp, sz, vp]),
             "qlora_check": (ctypes.c_int, [vp, vp]),
             "qlora_merge": (ctypes.c_int, [pq, vp, vp, i32, f32, vp, vp]),
+            "qlora_merge_dense": (ctypes.c_int, [vp, i64, i64, vp, vp, i32, f32, vp, vp]),
             "qlora_paged_alloc": (ctypes.c_int, [ctypes.c_size_t, ctypes.POINTER(ctypes.c_void_p)]),
             "qlora_paged_prefetch": (ctypes.c_int, [vp, ctypes.c_size_t, i32, vp]),
             "qlora_paged_free": (ctypes.c_int, [vp]),
@@ -404,6 +405,17 @@ def qlora_merge(q, A, B, alpha, out=None, stream=None):
     st = q.struct
     _ok(lib().qlora_merge(ctypes.byref(st), _ptr(A), _ptr(B), r, float(alpha), _ptr(out),
                           _stream(stream)), "qlora_merge")
+    return out
+
+
+def qlora_merge_dense(W, A, B, alpha, out=None, stream=None):
+    """bf16(W + (alpha / r) B A) for a dense bf16 W; out=W works in place, and
+    -alpha takes a merged adapter out again."""
+    r = A.shape[0]
+    rows, cols = W.shape
+    out = out if out is not None else torch.empty_like(W)
+    _ok(lib().qlora_merge_dense(_ptr(W), rows, cols, _ptr(A), _ptr(B), r, float(alpha), _ptr(out),
+                                _stream(stream)), "qlora_merge_dense")
     return out
 
 

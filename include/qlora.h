@@ -214,6 +214,16 @@ qlora_status qlora_linear_bwd_multi(const qlora_nf4* W, const void* A, const voi
 qlora_status qlora_merge(const qlora_nf4* W, const void* A, const void* B, int32_t r,
                          float alpha, void* W_out, void* stream);
 
+/* The same update on a dense bf16 weight: W_out = bf16(W_in + (alpha / r) B A),
+ * accumulated in fp32 and rounded once.  With -alpha it takes a merged
+ * adapter out again (unmerge), or, applied twice, moves a merged weight from
+ * one adapter to another.  Device buffers: W_in and W_out (rows x cols bf16,
+ * row-major; W_out may be W_in: in place), A (r x cols bf16), B (rows x r
+ * bf16), all 16-byte aligned.  Errors: QLORA_ERR_NULL, _ALIGN, _SHAPE (rows or
+ * cols < 1, cols % 8 != 0, r outside [1, 256], rows > 2^22), _CUDA. */
+qlora_status qlora_merge_dense(const void* W_in, int64_t rows, int64_t cols, const void* A,
+                               const void* B, int32_t r, float alpha, void* W_out, void* stream);
+
 /* One AdamW step (Adam with decoupled weight decay) over n adapter
  * parameters - the optimiser that updates only A and B ("QLoRA技术从入门到精
  * 通", section 3(3)).  For step >= 1, per element, g' = grad_scale * grad:

@@ -191,3 +191,14 @@ def test_multi_adapter_argument_errors_without_cuda():
     assert fwd(ids=P(0x50002)) == Q.QLORA_ERR_ALIGN
     assert fwd(n=3, r=5) == Q.QLORA_ERR_UNSUPPORTED  # 15 stacked ranks
     assert fwd(M=0, ids=None) == Q.QLORA_OK          # nothing to do: no launch
+
+
+def test_merge_dense_argument_errors_without_cuda():
+    L = Q.lib()
+    P = ctypes.c_void_p
+    w, a, b, o = P(0x20000), P(0x30000), P(0x40000), P(0x50000)
+    assert L.qlora_merge_dense(None, 8, 64, a, b, 8, 16.0, o, None) == Q.QLORA_ERR_NULL
+    assert L.qlora_merge_dense(w, 8, 60, a, b, 8, 16.0, o, None) == Q.QLORA_ERR_SHAPE   # cols % 8
+    assert L.qlora_merge_dense(w, 0, 64, a, b, 8, 16.0, o, None) == Q.QLORA_ERR_SHAPE
+    assert L.qlora_merge_dense(w, 8, 64, a, b, 257, 16.0, o, None) == Q.QLORA_ERR_SHAPE
+    assert L.qlora_merge_dense(w, 8, 64, P(0x30008), b, 8, 16.0, o, None) == Q.QLORA_ERR_ALIGN

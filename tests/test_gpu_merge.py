@@ -73,3 +73,45 @@ def test_merge_with_zero_b_is_the_compute_weight():
     torch.cuda.synchronize()
     ref = oracle.compute_weight(oracle.quantize(W.float().numpy(), 64, 256)).reshape(192, 512)
     assert np.array_equal(out.float().cpu().numpy(), ref)
+
+
+def _bound_ok(out, exact, base_abs, A, B, s, r):
+    # one bf16 ulp of the exact value plus the fp32 error of the rank-r sum
+    mag = base_abs + s * (np.abs(f64(B)) @ np.abs(f64(A)))
+    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(exact), 1e-38))) - 7)
+    return np.all(np.abs(f64(out) - exact) <= ulp + (r + 2) * 2.0 ** -24 * mag)
+
+
+def test_merge_dense_matches_oracle_and_works_in_place():
+    W = WL.randn((320, 1024), 0.02, 21, torch.bfloat16)
+    A = WL.randn((16, 1024), 0.25, 22, torch.bfloat16)
+    B = WL.randn((320, 16), 0.05, 23, torch.bfloat16)
+    Wd, Ad, Bd = W.to(DEV), A.to(DEV), B.to(DEV)
+    out = Q.qlora_merge_dense(Wd, Ad, Bd, 32.0)
+    inplace = Wd.clone()
+    Q.qlora_merge_dense(inplace, Ad, Bd, 32.0, out=inplace)
+    torch.cuda.synchronize()
+    exact = oracle.merge_weight(f64(W), f64(A), f64(B), 32.0)
+    assert _bound_ok(out, exact, np.abs(f64(W)), A, B, oracle.lora_scale(32.0, 16), 16)
+    assert torch.equal(out, inplace)
+
+
+def test_unmerge_restores_the_compute_weight():
+    # merge then merge_dense with -alpha: back to bf16(W_hat) up to the two roundings
+    W = WL.randn((256, 768), 0.02, 31, torch.bfloat16)
+    A = WL.randn((8, 768), 0.35, 32, torch.bfloat16)
+    B = WL.randn((256, 8), 0.05, 33, torch.bfloat16)
+    q = Q.qlora_quantize(W.to(DEV))
+    Ad, Bd = A.to(DEV), B.to(DEV)
+    merged = Q.qlora_merge(q, Ad, Bd, 16.0)
+    back = Q.qlora_merge_dense(merged, Ad, Bd, -16.0)
+    torch.cuda.synchronize()
+    # the unmerge step itself is the oracle's sum on the merged bf16 weight
+    exact = oracle.merge_weight(f64(merged), f64(A), f64(B), -16.0)
+    s = oracle.lora_scale(16.0, 8)
+    assert _bound_ok(back, exact, np.abs(f64(merged)), A, B, s, 8)
+    # and it lands next to the compute weight: within the two bf16 roundings
+    w_bf16 = oracle.compute_weight(oracle.quantize(W.float().numpy(), 64, 256)).reshape(256, 768)
+    upd = s * (np.abs(f64(B)) @ np.abs(f64(A)))
+    tol = 2.0 ** -7 * (np.abs(w_bf16) + upd) + 1e-30
+    assert np.all(np.abs(f64(back) - w_bf16) <= tol)
