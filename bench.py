@@ -531,8 +531,8 @@ def run_ours(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,.) tensors of the workload's shapes)",
-        "config": dict(workload_config(world),
-                       launch="one CUDA graph of the timed steps" if use_graph else "eager"),
+        "config": workload_config(world),
+        "launch": "one CUDA graph of the timed steps" if use_graph else "eager",
         "nf4_weight_gbs": round(2 * wb / (t_fwd + t_bwd) / 1e9, 1),
         "fwd_ms": round(t_fwd * 1e3, 4), "bwd_ms": round(t_bwd * 1e3, 4),
         "fwd_tflops": round(fwd_flops(M, N, K, r) / t_fwd / 1e12, 2),
