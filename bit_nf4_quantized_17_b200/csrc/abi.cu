@@ -4,7 +4,9 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <tuple>
 #include <vector>
 
 #include "internal.cuh"
@@ -28,6 +30,41 @@ struct Timing {
 };
 Timing g_timing;
 }  // namespace
+
+namespace {
+std::mutex g_setup_mu;
+std::map<std::tuple<int, const void*, int>, int> g_setup;  // (device, kernel, tag) -> value
+constexpr int kSmemTag = -1;
+}  // namespace
+
+bool qlora::cached_value(const void* func, int tag, int* value) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  std::lock_guard<std::mutex> lock(g_setup_mu);
+  const auto it = g_setup.find(std::make_tuple(dev, func, tag));
+  if (it == g_setup.end()) return false;
+  *value = it->second;
+  return true;
+}
+
+void qlora::store_value(const void* func, int tag, int value) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return;
+  std::lock_guard<std::mutex> lock(g_setup_mu);
+  g_setup[std::make_tuple(dev, func, tag)] = value;
+}
+
+qlora_status qlora::ensure_smem(const void* func, int bytes) {
+  int have = 0;
+  if (cached_value(func, kSmemTag, &have) && have >= bytes) return QLORA_OK;
+  if (cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+      cudaSuccess) {
+    (void)cudaGetLastError();
+    return QLORA_ERR_CUDA;
+  }
+  store_value(func, kSmemTag, bytes);
+  return QLORA_OK;
+}
 
 void qlora::count_launch(unsigned n) {
   g_launches.fetch_add(n, std::memory_order_relaxed);

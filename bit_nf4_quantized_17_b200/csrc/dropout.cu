@@ -111,13 +111,9 @@ qlora_status dropout_apply(const void* X, const uint8_t* mask, int64_t M, int64_
 qlora_status dropout_dx(void* dX, const float* V, int64_t ldv, const void* A, const uint8_t* mask,
                         int64_t M, int64_t K, int32_t r, float scale, cudaStream_t s) {
   const size_t smem = sizeof(__nv_bfloat16) * static_cast<size_t>(r) * kCols;
-  static bool configured = false;
-  if (!configured) {
-    if (cudaFuncSetAttribute(dropout_dx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(sizeof(__nv_bfloat16) * 256 * kCols)) != cudaSuccess)
-      return QLORA_ERR_CUDA;
-    configured = true;
-  }
+  const qlora_status cs = ensure_smem(reinterpret_cast<const void*>(dropout_dx_kernel),
+                                      static_cast<int>(sizeof(__nv_bfloat16) * 256 * kCols));
+  if (cs != QLORA_OK) return cs;
   const dim3 grid(static_cast<unsigned>(ceil_div(K, kCols)), static_cast<unsigned>(ceil_div(M, kRows)));
   if (grid.y > 65535) return QLORA_ERR_SHAPE;
   count_launch();

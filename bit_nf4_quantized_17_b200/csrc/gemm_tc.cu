@@ -595,14 +595,9 @@ qlora_status launch_tc(const CUtensorMap& a, const CUtensorMap& b, const CUtenso
                        cudaStream_t s) {
   const size_t smem = 1024 + static_cast<size_t>(STAGES) * p.stage_bytes +
                       CodesRing<BMODE, MT>::kBytes + 256;
-  static bool configured = false;
-  if (!configured) {
-    if (cudaFuncSetAttribute(tc_gemm_kernel<BMODE, STAGES, MT>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(232448)) != cudaSuccess)
-      return QLORA_ERR_CUDA;
-    configured = true;
-  }
+  const qlora_status cs =
+      ensure_smem(reinterpret_cast<const void*>(tc_gemm_kernel<BMODE, STAGES, MT>), 232448);
+  if (cs != QLORA_OK) return cs;
   count_launch();
   constexpr int kind = BMODE == B_TMA_K   ? QLORA_KERNEL_LORA_GEMM
                        : BMODE == B_DQ_K ? QLORA_KERNEL_FUSED_FWD

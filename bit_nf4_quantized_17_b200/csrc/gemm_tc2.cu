@@ -331,13 +331,9 @@ template <int BMODE>
 qlora_status launch_tc2(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& ma2,
                         const CUtensorMap& mb2, const Tc2Args& p, const LevelTable& t,
                         int64_t m_pairs, int64_t n_tiles, cudaStream_t s) {
-  static bool configured = false;
-  if (!configured) {
-    if (cudaFuncSetAttribute(tc2_fused_kernel<BMODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kSmemBytes) != cudaSuccess)
-      return QLORA_ERR_CUDA;
-    configured = true;
-  }
+  const qlora_status cs = ensure_smem(reinterpret_cast<const void*>(tc2_fused_kernel<BMODE>),
+                                      kSmemBytes);
+  if (cs != QLORA_OK) return cs;
   if (m_pairs < 1 || 2 * m_pairs > 0x7fffffff || n_tiles < 1 || n_tiles > 65535)
     return QLORA_ERR_SHAPE;
   cudaLaunchConfig_t cfg = {};

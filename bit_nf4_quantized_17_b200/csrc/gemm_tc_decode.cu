@@ -383,13 +383,9 @@ qlora_status tc_decode_forward(const QView& w, const LevelTable& t, const void* 
   p.out_elems = M * N;
   p.cluster = splits;
   p.st = st;
-  static bool configured = false;
-  if (!configured) {
-    if (cudaFuncSetAttribute(tc_decode_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kSmemBytes) != cudaSuccess)
-      return QLORA_ERR_CUDA;
-    configured = true;
-  }
+  const qlora_status cs =
+      ensure_smem(reinterpret_cast<const void*>(tc_decode_fwd_kernel), kSmemBytes);
+  if (cs != QLORA_OK) return cs;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>(ceil_div(N, 128)), static_cast<unsigned>(splits), 1);
   cfg.blockDim = dim3(kThreads, 1, 1);

@@ -205,16 +205,17 @@ qlora_status gemv_dgrad(const QView& w, const LevelTable& t, const void* dY, int
   cfg.numAttrs = 1;
   // as many row chunks as keep every cluster resident at once (one wave),
   // within the workspace's bound
-  static int resident[2] = {0, 0};
-  int& res = resident[M == 1 ? 0 : 1];
-  if (res == 0) {
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-      return QLORA_ERR_CUDA;
+  const void* fn = reinterpret_cast<const void*>(kernel);
+  const qlora_status cs = ensure_smem(fn, static_cast<int>(smem));
+  if (cs != QLORA_OK) return cs;
+  int res = 0;
+  if (!cached_value(fn, 0, &res)) {
     cfg.gridDim = dim3(kCluster, 1, 1);
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n < 1) n = 1;
-    res = n;
+    if (cudaOccupancyMaxActiveClusters(&res, kernel, &cfg) != cudaSuccess || res < 1) {
+      (void)cudaGetLastError();
+      res = 1;
+    }
+    store_value(fn, 0, res);
   }
   int C = (res / nkg) * kCluster;
   if (C > max_chunks(K)) C = max_chunks(K);

@@ -39,6 +39,13 @@ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 // abi.cu: every kernel launch site calls this once per launch.
 void count_launch(unsigned n = 1);
+// Per-device, thread-safe launch setup.  ensure_smem raises `func`'s dynamic
+// shared-memory limit on the current device to at least `bytes` (once per
+// device).  cached_value / store_value keep a per-device integer for `func`
+// under `tag` (resident CTA or cluster counts measured once).
+qlora_status ensure_smem(const void* func, int bytes);
+bool cached_value(const void* func, int tag, int* value);
+void store_value(const void* func, int tag, int value);
 
 // abi.cu: kernel timing hook.  A launch site of a timed kind calls it with
 // start = true just before its launch and start = false just after; both are

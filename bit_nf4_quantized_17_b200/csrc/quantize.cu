@@ -390,23 +390,23 @@ qlora_status launch_blocks(int bs, const T* w, int64_t n, const LevelTable& t, u
   if (!make_cell_lut(t, &cells)) return QLORA_ERR_UNSUPPORTED;
   const int64_t chunks = ceil_div(n, bs <= 512 ? 16 : 32);
   // persistent grid: as many CTAs as fit on the device at once
-  static int resident[2][5] = {};
-  const int ti = sizeof(T) == 4 ? 0 : 1, bi = __builtin_ctz(bs) - 6;
-  if (!resident[ti][bi]) {
+  const void* fn = bs == 64    ? reinterpret_cast<const void*>(quantize_blocks_kernel<T, 64>)
+                   : bs == 128 ? reinterpret_cast<const void*>(quantize_blocks_kernel<T, 128>)
+                   : bs == 256 ? reinterpret_cast<const void*>(quantize_blocks_kernel<T, 256>)
+                   : bs == 512 ? reinterpret_cast<const void*>(quantize_blocks_kernel<T, 512>)
+                               : reinterpret_cast<const void*>(quantize_blocks_kernel<T, 1024>);
+  int resident = 0;
+  if (!cached_value(fn, 0, &resident)) {
     int dev = 0, sms = 148, per_sm = 0;
-    const void* fn = bs == 64    ? reinterpret_cast<const void*>(quantize_blocks_kernel<T, 64>)
-                     : bs == 128 ? reinterpret_cast<const void*>(quantize_blocks_kernel<T, 128>)
-                     : bs == 256 ? reinterpret_cast<const void*>(quantize_blocks_kernel<T, 256>)
-                     : bs == 512 ? reinterpret_cast<const void*>(quantize_blocks_kernel<T, 512>)
-                                 : reinterpret_cast<const void*>(quantize_blocks_kernel<T, 1024>);
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, 256, 0) != cudaSuccess ||
         per_sm < 1)
       return QLORA_ERR_CUDA;
-    resident[ti][bi] = sms * per_sm;
+    resident = sms * per_sm;
+    store_value(fn, 0, resident);
   }
-  const int grid = grid_for(chunks, 256, resident[ti][bi]);
+  const int grid = grid_for(chunks, 256, resident);
   count_launch();
   timing_mark(QLORA_KERNEL_QUANTIZE, s, true);
   switch (bs) {
