@@ -28,6 +28,11 @@
  *     qlora_paged_free, whose whole job is that.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
  *     stream-ordered and asynchronous: they return after enqueueing work.
+ *     The backward pass of larger batches forks its dA/dB work onto a second,
+ *     library-owned stream (one per host thread and device, created on first
+ *     use and kept until the process exits) and joins it back before it
+ *     returns, so the call stays ordered on `stream` and can be captured in a
+ *     CUDA graph.
  *   - Argument errors are found on the host and returned before any launch.
  *     Errors found on the device (a non-finite weight, a bounded wait that
  *     gave up) are written to a status word at the start of the workspace;
