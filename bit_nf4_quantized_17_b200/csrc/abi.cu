@@ -9,9 +9,12 @@
 #include <tuple>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "internal.cuh"
 #include "kernels.cuh"
 #include "linear.cuh"
+#include "tc_ptx.cuh"
 
 using namespace qlora;
 
@@ -166,6 +169,32 @@ size_t quantize_workspace(int64_t n, int32_t bs, int32_t dq) {
 
 }  // namespace
 
+namespace {
+// An NVTX range around an ABI call, so that profiles show the library's calls
+// (free when no tool is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
+// One CTA waits on an mbarrier that nothing completes, with the library's
+// bounded wait, and reports the timeout the way the real kernels do.
+__global__ void timeout_selftest_kernel(long long limit, DeviceStatus* st) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(&bar, 1);
+    abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+  if (!ptx::mbar_wait(&bar, 0, limit, &abort_flag) && threadIdx.x == 0)
+    report(st, QLORA_ERR_DEVICE_TIMEOUT, 900u);
+}
+}  // namespace
+
 extern "C" {
 
 const char* qlora_status_string(qlora_status s) {
@@ -214,6 +243,7 @@ qlora_status qlora_nf4_sizes(int64_t rows, int64_t cols, int32_t blocksize, int3
 
 qlora_status qlora_quantize(const void* W, int32_t w_dtype, const qlora_nf4* q, void* workspace,
                             size_t workspace_bytes, void* stream) {
+  const NvtxRange nvtx("qlora_quantize");
   if (!q || !W || !workspace) return QLORA_ERR_NULL;
   qlora_status st = check_nf4_shape(*q);
   if (st != QLORA_OK) return st;
@@ -228,6 +258,7 @@ qlora_status qlora_quantize(const void* W, int32_t w_dtype, const qlora_nf4* q, 
 }
 
 qlora_status qlora_dequantize(const qlora_nf4* q, void* W_out, int32_t out_dtype, void* stream) {
+  const NvtxRange nvtx("qlora_dequantize");
   if (!q || !W_out) return QLORA_ERR_NULL;
   qlora_status st = check_nf4_shape(*q);
   if (st != QLORA_OK) return st;
@@ -242,6 +273,7 @@ qlora_status qlora_dequantize(const qlora_nf4* q, void* W_out, int32_t out_dtype
 qlora_status qlora_adamw(float* param, void* param_bf16, const float* grad, float* m, float* v,
                          int64_t n, int32_t step, float lr, float beta1, float beta2, float eps,
                          float weight_decay, float grad_scale, void* stream) {
+  const NvtxRange nvtx("qlora_adamw");
   if (n < 0 || step < 1) return QLORA_ERR_SHAPE;
   if (n == 0) return QLORA_OK;
   if (!param || !grad || !m || !v) return QLORA_ERR_NULL;
@@ -286,6 +318,7 @@ qlora_status qlora_paged_free(void* ptr) {
 
 qlora_status qlora_merge(const qlora_nf4* W, const void* A, const void* B, int32_t r,
                          float alpha, void* W_out, void* stream) {
+  const NvtxRange nvtx("qlora_merge");
   if (!W || !A || !B || !W_out) return QLORA_ERR_NULL;
   qlora_status st = check_nf4_shape(*W);
   if (st != QLORA_OK) return st;
@@ -300,6 +333,7 @@ qlora_status qlora_merge(const qlora_nf4* W, const void* A, const void* B, int32
 
 qlora_status qlora_merge_dense(const void* W_in, int64_t rows, int64_t cols, const void* A,
                                const void* B, int32_t r, float alpha, void* W_out, void* stream) {
+  const NvtxRange nvtx("qlora_merge_dense");
   if (!W_in || !A || !B || !W_out) return QLORA_ERR_NULL;
   if (rows < 1 || cols < 1 || cols % 8 != 0 || r < 1 || r > 256 || rows > (int64_t(1) << 22))
     return QLORA_ERR_SHAPE;
@@ -339,6 +373,7 @@ static qlora_status check_linear(const qlora_nf4* W, const void* A, const void* 
 qlora_status qlora_linear_fwd(const qlora_nf4* W, const void* A, const void* B, int32_t r,
                               float alpha, const void* X, int64_t M, void* Y, float* U_save,
                               void* workspace, size_t workspace_bytes, void* stream) {
+  const NvtxRange nvtx("qlora_linear_fwd");
   qlora_status st = check_linear(W, A, B, r, M, X, workspace, workspace_bytes, false);
   if (st != QLORA_OK) return st;
   if (M == 0) return QLORA_OK;
@@ -352,6 +387,7 @@ qlora_status qlora_linear_bwd(const qlora_nf4* W, const void* A, const void* B, 
                               float alpha, const void* X, const float* U, const void* dY,
                               int64_t M, void* dX, float* dA, float* dB, int32_t accumulate,
                               void* workspace, size_t workspace_bytes, void* stream) {
+  const NvtxRange nvtx("qlora_linear_bwd");
   qlora_status st = check_linear(W, A, B, r, M, X, workspace, workspace_bytes, true);
   if (st != QLORA_OK) return st;
   if ((M > 0 && !dY) || !dA || !dB) return QLORA_ERR_NULL;
@@ -408,6 +444,7 @@ qlora_status qlora_linear_fwd_ex(const qlora_nf4* W, const void* A, const void* 
                                  float alpha, const qlora_adapter_opts* opts, const void* X,
                                  int64_t M, void* Y, float* U_save, void* workspace,
                                  size_t workspace_bytes, void* stream) {
+  const NvtxRange nvtx("qlora_linear_fwd_ex");
   if (!W) return QLORA_ERR_NULL;
   LoraOpts o{};
   int32_t rt = 0;
@@ -427,6 +464,7 @@ qlora_status qlora_linear_bwd_ex(const qlora_nf4* W, const void* A, const void* 
                                  const float* U, const void* dY, int64_t M, void* dX, float* dA,
                                  float* dB, int32_t accumulate, void* workspace,
                                  size_t workspace_bytes, void* stream) {
+  const NvtxRange nvtx("qlora_linear_bwd_ex");
   if (!W) return QLORA_ERR_NULL;
   LoraOpts o{};
   int32_t rt = 0;
@@ -475,6 +513,17 @@ qlora_status qlora_linear_bwd_multi(const qlora_nf4* W, const void* A, const voi
   if (M > 0 && !adapter) return QLORA_ERR_NULL;
   return qlora_linear_bwd_ex(W, A, B, r, alpha, &x, X, U, dY, M, dX, dA, dB, accumulate,
                              workspace, workspace_bytes, stream);
+}
+
+qlora_status qlora_selftest_timeout(int64_t limit_cycles, void* workspace, void* stream) {
+  if (!workspace) return QLORA_ERR_NULL;
+  if (limit_cycles < 1 || limit_cycles > (int64_t(1) << 32)) return QLORA_ERR_SHAPE;
+  if (!aligned16(workspace)) return QLORA_ERR_ALIGN;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  count_launch();
+  timeout_selftest_kernel<<<1, 32, 0, s>>>(static_cast<long long>(limit_cycles),
+                                           static_cast<DeviceStatus*>(workspace));
+  return after_launch("timeout_selftest", s);
 }
 
 qlora_status qlora_check(void* workspace, void* stream) {

@@ -100,6 +100,7 @@ def lib():
             "qlora_linear_bwd_ex": (ctypes.c_int, [pq, vp, vp, i32, f32, po, vp, vp, vp, i64, vp,
                                                    vp, vp, i32, vp, sz, vp]),
             "qlora_check": (ctypes.c_int, [vp, vp]),
+            "qlora_selftest_timeout": (ctypes.c_int, [i64, vp, vp]),
             "qlora_merge": (ctypes.c_int, [pq, vp, vp, i32, f32, vp, vp]),
             "qlora_merge_dense": (ctypes.c_int, [vp, i64, i64, vp, vp, i32, f32, vp, vp]),
             "qlora_paged_alloc": (ctypes.c_int, [ctypes.c_size_t, ctypes.POINTER(ctypes.c_void_p)]),
@@ -479,6 +480,12 @@ def qlora_timing_end():
     n = (ctypes.c_int32 * QLORA_KERNEL_KINDS)()
     _ok(lib().qlora_timing_end(ms, n), "qlora_timing_end")
     return {k: (float(ms[k]), int(n[k])) for k in range(QLORA_KERNEL_KINDS)}
+
+
+def qlora_selftest_timeout(limit_cycles, workspace, stream=None):
+    """Enqueue the library's bounded-wait failure path on purpose (see the header)."""
+    _ok(lib().qlora_selftest_timeout(int(limit_cycles), _ptr(workspace), _stream(stream)),
+        "qlora_selftest_timeout")
 
 
 def qlora_check(workspace, stream=None):

@@ -302,6 +302,14 @@ qlora_status qlora_paged_alloc(size_t bytes, void** ptr);
 qlora_status qlora_paged_prefetch(void* ptr, size_t bytes, int32_t to_device, void* stream);
 qlora_status qlora_paged_free(void* ptr);
 
+/* Diagnostic of the failure path: one CTA waits, with the library's bounded
+ * wait, on an mbarrier that nothing completes, gives up after `limit_cycles`
+ * clock cycles (1 .. 2^32) and writes QLORA_ERR_DEVICE_TIMEOUT to the status
+ * word of `workspace` (at least 256 bytes), as the library's kernels do when
+ * one of their waits runs out.  qlora_check then returns that code and clears
+ * it; the context stays usable.  Errors: QLORA_ERR_NULL, _SHAPE, _ALIGN, _CUDA. */
+qlora_status qlora_selftest_timeout(int64_t limit_cycles, void* workspace, void* stream);
+
 /* Synchronise `stream`, then return and clear the device status word that
  * calls given this workspace wrote (QLORA_OK if none). */
 qlora_status qlora_check(void* workspace, void* stream);

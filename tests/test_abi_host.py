@@ -202,3 +202,12 @@ def test_merge_dense_argument_errors_without_cuda():
     assert L.qlora_merge_dense(w, 0, 64, a, b, 8, 16.0, o, None) == Q.QLORA_ERR_SHAPE
     assert L.qlora_merge_dense(w, 8, 64, a, b, 257, 16.0, o, None) == Q.QLORA_ERR_SHAPE
     assert L.qlora_merge_dense(w, 8, 64, P(0x30008), b, 8, 16.0, o, None) == Q.QLORA_ERR_ALIGN
+
+
+def test_timeout_selftest_argument_errors_without_cuda():
+    L = Q.lib()
+    P = ctypes.c_void_p
+    assert L.qlora_selftest_timeout(1000, None, None) == Q.QLORA_ERR_NULL
+    assert L.qlora_selftest_timeout(0, P(0x10000), None) == Q.QLORA_ERR_SHAPE
+    assert L.qlora_selftest_timeout(2 ** 33, P(0x10000), None) == Q.QLORA_ERR_SHAPE
+    assert L.qlora_selftest_timeout(1000, P(0x10004), None) == Q.QLORA_ERR_ALIGN
