@@ -108,3 +108,24 @@ def test_bucket_views_are_aligned_and_disjoint():
     assert torch.count_nonzero(bk.dB) == 0
     with pytest.raises(ValueError):
         dp.token_shard(10, 2, 2)
+
+
+def test_adapter_optimizer_layout_matches_the_gradient_bucket():
+    # AdapterAdamW keeps A and B (fp32 master and bf16 views) at the offsets of
+    # GradBucket, so that one flat AdamW step pairs every parameter with its
+    # gradient; checked on the host (no kernel runs here)
+    from bit_nf4_quantized_17_b200.optim import AdapterAdamW
+
+    r, d_in, d_out = 8, 200, 72
+    A = torch.randn(r, d_in).to(torch.bfloat16)
+    B = torch.randn(d_out, r).to(torch.bfloat16)
+    opt = AdapterAdamW(A, B, lr=1e-3)
+    bucket = opt.grad_bucket()
+    assert opt.master.shape == bucket.flat.shape
+    assert torch.equal(opt.A, A) and torch.equal(opt.B, B)
+    na = r * d_in
+    assert torch.equal(opt.master[:na].view(r, d_in), A.float())
+    assert torch.equal(opt.master[bucket.off_b:bucket.off_b + d_out * r].view(d_out, r), B.float())
+    assert opt.A.data_ptr() == opt.bf16.data_ptr()
+    assert opt.B.data_ptr() == opt.bf16.data_ptr() + 2 * bucket.off_b
+    assert bucket.dB.data_ptr() == bucket.flat.data_ptr() + 4 * bucket.off_b
