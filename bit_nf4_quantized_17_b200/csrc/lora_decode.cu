@@ -88,17 +88,17 @@ __device__ __forceinline__ void store_rank(const RankOut& o, int m, int j, float
   }
 }
 
-// Sum the per-CTA partials red[w][m] (8 ranks x MM tokens) over the cluster's
+// Sum the per-CTA partials red[w][m] (JB ranks x MM tokens) over the cluster's
 // CTAs in rank order and store; CTA q of the cluster writes the items
 // t = q, q + nrank, ... of the 8 MM, and every CTA keeps its shared memory
 // until the others have read it.
-template <int MM>
-__device__ __forceinline__ void cluster_finish(const float (&red)[8][MM], const RankOut& o, int M,
+template <int MM, int JB>
+__device__ __forceinline__ void cluster_finish(const float (&red)[JB][MM], const RankOut& o, int M,
                                                int jb) {
   ptx::cluster_sync();
   const int nrank = static_cast<int>(gridDim.x);  // the cluster spans the grid's x dimension
   for (int t = static_cast<int>(ptx::cluster_ctarank()) + nrank * static_cast<int>(threadIdx.x);
-       t < 8 * MM; t += nrank * static_cast<int>(blockDim.x)) {
+       t < JB * MM; t += nrank * static_cast<int>(blockDim.x)) {
     const int w = t / MM, m = t % MM;
     float x[kMaxChunks];
 #pragma unroll
@@ -108,7 +108,7 @@ __device__ __forceinline__ void cluster_finish(const float (&red)[8][MM], const 
 #pragma unroll
     for (int q = 0; q < kMaxChunks; ++q)
       if (q < nrank) v += x[q];
-    if (m < M) store_rank(o, m, 8 * jb + w, v);
+    if (m < M) store_rank(o, m, JB * jb + w, v);
   }
   ptx::cluster_sync();
 }
@@ -163,60 +163,71 @@ rank_down_kernel(const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __res
     }
   }
   warp_sum_store<MM>(acc, lane, red[warp]);
-  cluster_finish<MM>(red, o, M, jb);
+  cluster_finish<MM, 8>(red, o, M, jb);
 }
 
 // V = dY B.  CTA (c, jb): rows [c len, (c + 1) len) of B, rank columns
-// 8 jb .. 8 jb + 7 (16 bytes of each row); thread t takes rows t, t + 256, ...,
-// loading kAhead rows (B and the tokens' dY values) before using them.
+// JB jb .. JB jb + JB - 1 (2 JB bytes of each row); thread t takes rows t,
+// t + 256, ..., loading kAhead rows (B and the tokens' dY values) before using
+// them.  Wide token counts take 4-rank blocks: half the accumulators per
+// thread, twice the CTAs.
 template <int MM>
 __global__ void __launch_bounds__(kThreads)
 rank_v_kernel(const __nv_bfloat16* __restrict__ dY, const __nv_bfloat16* __restrict__ B, int M,
               int64_t N, int len, RankOut o) {
+  constexpr int JB = MM >= 8 ? 4 : 8;
   constexpr int kAhead = MM >= 8 ? 2 : 4;
-  __shared__ float wred[8][MM * 8];
-  __shared__ float red[8][MM];
+  __shared__ float wred[8][MM * JB];
+  __shared__ float red[JB][MM];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int jb = blockIdx.y;
-  const bool real = 8 * jb < o.r;  // r is a multiple of 8: a block is all ranks or all padding
+  const bool real = JB * jb < o.r;  // r is a multiple of 8: a block is all ranks or all padding
   const int64_t c0 = static_cast<int64_t>(blockIdx.x) * len;
   const int64_t c1 = (c0 + len < N) ? c0 + len : N;
-  float acc[MM * 8];  // [m][q]
+  float acc[MM * JB];  // [m][q]
 #pragma unroll
-  for (int e = 0; e < MM * 8; ++e) acc[e] = 0.0f;
+  for (int e = 0; e < MM * JB; ++e) acc[e] = 0.0f;
   if (real) {
     for (int64_t n0 = c0 + threadIdx.x; n0 < c1; n0 += kAhead * kThreads) {
-      uint4 bv[kAhead];
+      float bf[kAhead][JB];
       float dy[kAhead][MM];
 #pragma unroll
       for (int u = 0; u < kAhead; ++u) {
         const int64_t n = n0 + static_cast<int64_t>(u) * kThreads;
         const bool in = n < c1;
-        bv[u] = in ? *reinterpret_cast<const uint4*>(B + n * o.r + 8 * jb) : make_uint4(0u, 0u, 0u, 0u);
+        if constexpr (JB == 8) {
+          const uint4 v = in ? *reinterpret_cast<const uint4*>(B + n * o.r + 8 * jb)
+                             : make_uint4(0u, 0u, 0u, 0u);
+          bf16x8_to_f32(v, bf[u]);
+        } else {
+          const uint2 v = in ? *reinterpret_cast<const uint2*>(B + n * o.r + 4 * jb)
+                             : make_uint2(0u, 0u);
+          bf[u][0] = __uint_as_float(v.x << 16);
+          bf[u][1] = __uint_as_float(v.x & 0xffff0000u);
+          bf[u][2] = __uint_as_float(v.y << 16);
+          bf[u][3] = __uint_as_float(v.y & 0xffff0000u);
+        }
 #pragma unroll
         for (int m = 0; m < MM; ++m) dy[u][m] = (in && m < M) ? __bfloat162float(dY[m * N + n]) : 0.0f;
       }
 #pragma unroll
-      for (int u = 0; u < kAhead; ++u) {
-        float b[8];
-        bf16x8_to_f32(bv[u], b);
+      for (int u = 0; u < kAhead; ++u)
 #pragma unroll
         for (int m = 0; m < MM; ++m)
 #pragma unroll
-          for (int q = 0; q < 8; ++q) acc[8 * m + q] = fmaf(dy[u][m], b[q], acc[8 * m + q]);
-      }
+          for (int q = 0; q < JB; ++q) acc[JB * m + q] = fmaf(dy[u][m], bf[u][q], acc[JB * m + q]);
     }
   }
   // sum over the CTA's threads: the lanes of each warp, then the 8 warps in order
-  warp_sum_store<MM * 8>(acc, lane, wred[warp]);
+  warp_sum_store<MM * JB>(acc, lane, wred[warp]);
   __syncthreads();
-  for (int t = threadIdx.x; t < 8 * MM; t += kThreads) {
+  for (int t = threadIdx.x; t < JB * MM; t += kThreads) {
     const int q = t / MM, m = t % MM;
     float v = 0.0f;
-    for (int w = 0; w < 8; ++w) v += wred[w][8 * m + q];
+    for (int w = 0; w < 8; ++w) v += wred[w][JB * m + q];
     red[q][m] = v;
   }
-  cluster_finish<MM>(red, o, M, jb);
+  cluster_finish<MM, JB>(red, o, M, jb);
 }
 
 int tokens_pad(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : M <= 8 ? 8 : 16; }
@@ -280,7 +291,7 @@ qlora_status rank_v(const void* dY, const void* B, int M, int64_t N, int32_t spa
   if (M < 1 || M > kSmallM || o.r % 8 != 0) return QLORA_ERR_UNSUPPORTED;
   int chunks, len;
   chunking(N, &chunks, &len);
-  const int jblocks = ceil_div(span, 8);
+  const int jblocks = ceil_div(span, tokens_pad(M) >= 8 ? 4 : 8);  // the kernel's JB
   qlora_status st;
   switch (tokens_pad(M)) {
     case 1: st = launch_cluster(rank_v_kernel<1>, chunks, jblocks, s, dY, B, M, N, len, o); break;
