@@ -5,14 +5,21 @@
 // Backward (same pages, 6 and 3(3)): V = dY B, dX = dY W + s V A,
 // dB = s dY^T U, dA = s V^T X; no gradient for W.
 //
-// Tensor-core path (tcgen05, gemm_tc.cu), taken when d_out % 8 == 0 and
-// r % 8 == 0 (TMA needs 16-byte row strides); decode-sized M splits the fused
-// kernels over the contraction so that every SM streams weights:
-//   forward   U-GEMM (split-K) -> reduce (U fp32, sU bf16) -> fused
-//             dequant GEMM with the LoRA term as extra K stages          3 launches
-//   backward  U^T (transpose of the given U, or U-GEMM + reduce), B^T,
-//             V-GEMM -> reduce (sV, V^T), fused dequant dX GEMM,
-//             dB-GEMM -> reduce, dA-GEMM -> reduce                      8-9 launches
+// Tensor-core paths (tcgen05), taken when d_out % 8 == 0 and r % 8 == 0 (TMA
+// needs 16-byte row strides):
+//   M <= 16   forward   U = X A^T in one cluster-reduced launch (U_save, sU),
+//                       then the decode kernel with W in TMEM; its contraction
+//                       splits are summed in their cluster             2 launches
+//             backward  V = dY B in one launch (V, sV), dX by the CUDA-core GEMV
+//                       (M <= 2, clustered row chunks + one reduce) or by the
+//                       single-CTA fused kernel (split + reduce), then dB and dA
+//   M > 16    forward   U-GEMM (split-K) -> reduce (U fp32, sU bf16) -> fused
+//                       dequant GEMM (CTA pairs for large M) with the LoRA term
+//                       as extra K stages                                 3 launches
+//             backward  B^T, V-GEMM -> reduce (sV, V^T), fused dX GEMM on the
+//                       caller's stream; U^T, dB-GEMM -> reduce, dA-GEMM ->
+//                       reduce on a second stream that joins back        8-9 launches
+// Several adapters per batch and LoRA dropout use the same kernels (LoraOpts).
 // Other shapes take the CUDA-core contraction of gemm_simt.cu.
 #include <algorithm>
 
