@@ -12,13 +12,16 @@
 // N = 16) reads the token tile from shared memory (TMA, 128B swizzle).  The
 // LoRA term runs as extension stages with both operands in shared memory
 // (B's rows as A, sU as B).  The contraction is split over CTAs when the
-// rows alone give too few; the fp32 partials are summed by splitk_reduce.
+// rows alone give too few; the splits of a row tile form a thread-block
+// cluster and sum their fp32 tiles in shared memory, in split order, before
+// the one bf16 store of Y.
 //
-// Roles (320 threads, two CTAs per SM): warp 0 TMA producer, warp 1 TMEM
-// owner and MMA issuer, warps 2-9 two dequant groups of four warps (group g
-// takes k-tiles i % 2 == g; warp w writes TMEM lanes 32 (w % 4) .. + 31, so
-// warps 2-5 and 6-9 each cover all 128 lanes), group 0 drains the
-// accumulator.  Every wait is bounded.
+// Roles (320 threads, two CTAs per SM): warp 0 TMA producer (up to 8 stages
+// of token tile + codes in flight), warp 1 TMEM owner and MMA issuer, warps
+// 2-9 two dequant groups of four warps (group g takes k-tiles i % 2 == g and
+// writes one of 4 TMEM slots, freed by the commit of their MMAs; warp w writes
+// TMEM lanes 32 (w % 4) .. + 31, so warps 2-5 and 6-9 each cover all 128
+// lanes), group 0 drains the accumulator.  Every wait is bounded.
 #include <cudaTypedefs.h>
 
 #include "internal.cuh"
