@@ -228,7 +228,7 @@ def kernel_rooflines(kt, M, N, K, r, peaks):
     return out
 
 
-def time_decode(Q, WL, dev, peaks, steps=30, warmup=5):
+def time_decode(Q, WL, dev, peaks, steps=50, warmup=5):
     """Decode-shaped gate/up linear (11008 x 4096, r = 64) at M = 1 and 16:
     forward + backward, 8 rotating weight copies (8 x 23 MB > L2)."""
     shape = WL.WORKLOADS["mlp_11008"].linears[0]
