@@ -475,39 +475,68 @@ def run_ours(args):
                 "algorithmic_per_launch": d["algorithmic_per_launch"],
                 "peak_kind": d["peak_kind"]}
 
-    # end to end: host (pinned) inputs copied in, results copied out, every step
+    # end to end: every step copies its inputs in from pinned host memory and
+    # its results out to pinned host memory.  The copies run on their own
+    # streams (one per direction), so that the next step's upload and the
+    # previous step's download overlap this step's compute; two device slots
+    # alternate, each reused only after its step's results have left.
     e2e = None
     if not args.no_e2e:
-        s = sets[0]
-        host = {k: getattr(s, k).cpu().pin_memory() for k in ("W", "A", "B", "X", "dY")}
-        outs = {k: torch.empty_like(getattr(s, k), device="cpu").pin_memory()
-                for k in ("Y", "dX", "dA", "dB")}
-        h2d = sum(t.numel() * t.element_size() for t in host.values())
-        d2h = sum(t.numel() * t.element_size() for t in outs.values())
+        in_keys, out_keys = ("W", "A", "B", "X", "dY"), ("Y", "dX", "dA", "dB")
+        slots = sets[:2]
+        host_in = [{k: getattr(sl, k).cpu().pin_memory() for k in in_keys} for sl in slots]
+        host_out = [{k: torch.empty_like(getattr(sl, k), device="cpu").pin_memory()
+                     for k in out_keys} for sl in slots]
+        h2d = sum(t.numel() * t.element_size() for t in host_in[0].values())
+        d2h = sum(t.numel() * t.element_size() for t in host_out[0].values())
+        compute = torch.cuda.current_stream()
+        up, down = torch.cuda.Stream(), torch.cuda.Stream()
 
-        def e2e_step():
-            for k, t in host.items():
-                getattr(s, k).copy_(t, non_blocking=True)
-            run_step(s, shape, Q, world=world)
-            for k, t in outs.items():
-                t.copy_(getattr(s, k), non_blocking=True)
+        def e2e_steps(n):
+            up.wait_stream(compute)
+            done_compute, done_down = [], []
+            for i in range(n):
+                j = i % 2
+                sl = slots[j]
+                with torch.cuda.stream(up):
+                    if i >= 2:  # the slot's previous step has computed and downloaded
+                        up.wait_event(done_compute[i - 2])
+                        up.wait_event(done_down[i - 2])
+                    for k, t in host_in[j].items():
+                        getattr(sl, k).copy_(t, non_blocking=True)
+                    uploaded = torch.cuda.Event()
+                    uploaded.record(up)
+                compute.wait_event(uploaded)
+                run_step(sl, shape, Q, world=world)
+                ev = torch.cuda.Event()
+                ev.record(compute)
+                done_compute.append(ev)
+                with torch.cuda.stream(down):
+                    down.wait_event(ev)
+                    for k, t in host_out[j].items():
+                        t.copy_(getattr(sl, k), non_blocking=True)
+                    ev2 = torch.cuda.Event()
+                    ev2.record(down)
+                    done_down.append(ev2)
+            compute.wait_stream(up)
+            compute.wait_stream(down)
 
-        for _ in range(args.warmup):
-            e2e_step()
+        e2e_steps(args.warmup)
         torch.cuda.synchronize()
         barrier(world)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(args.steps):
-            e2e_step()
-        e1.record()
+        e0.record(compute)
+        e2e_steps(args.steps)
+        e1.record(compute)
         torch.cuda.synchronize()
         e2e_ms = dp.max_over_ranks(e0.elapsed_time(e1), dev) / args.steps
         e2e = {"value": round(flops_step * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
                "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h,
-               "path": "pinned host -> device copies, qlora_quantize + qlora_linear_fwd + "
-                       "qlora_linear_bwd through the C ABI, device -> pinned host copies"}
+               "path": "pinned host -> device copies (upload stream), qlora_quantize + "
+                       "qlora_linear_fwd + qlora_linear_bwd through the C ABI, device -> pinned "
+                       "host copies (download stream); two device slots, so that copies of "
+                       "neighbouring steps overlap the compute"}
 
     decode = None
     if rank == 0 and world == 1 and not args.no_decode:
