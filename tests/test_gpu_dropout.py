@@ -115,3 +115,29 @@ def test_keep_mask_helper_rate():
     kept = int(np.unpackbits(m.cpu().numpy(), bitorder="little").sum())
     frac = kept / (512 * 4096)
     assert abs(frac - 0.9) < 0.005
+
+
+@pytest.mark.parametrize("M", [13, 700])
+def test_recomputed_u_matches_the_saved_one(M):
+    # the backward without U recomputes it from X (.) D with the same scale and
+    # adapter mask as the forward: the gradients are bit-identical
+    N, K, r, n, p = 512, 1024, 8, 2, 0.1
+    shape = WL.LinearShape(N, K, n * r, 2.0 * r)
+    inp = WL.linear_inputs(shape, M, 300 + M)
+    q = Q.qlora_quantize(inp["W"].to(DEV))
+    A = WL.randn((n * r, K), 0.3, 5, torch.bfloat16).to(DEV)
+    B = WL.randn((N, n * r), 0.05, 6, torch.bfloat16).to(DEV)
+    X, dY = inp["X"].to(DEV), inp["dY"].to(DEV)
+    ids = torch.from_numpy(np.random.default_rng(M).integers(-1, n, M).astype(np.int32)).to(DEV)
+    md = torch.from_numpy(_mask(M, K, p, 9)).to(DEV)
+    xdrop = torch.empty_like(X)
+    U = torch.empty((M, n * r), dtype=torch.float32, device=DEV)
+    Q.qlora_linear_fwd_ex(q, A, B, r, 2.0 * r, X, adapter=ids, p=p, keep_mask=md, x_drop=xdrop,
+                          U_save=U, check=True)
+    g_saved = Q.qlora_linear_bwd_ex(q, A, B, r, 2.0 * r, X, U, dY, adapter=ids, p=p,
+                                    keep_mask=md, x_drop=xdrop, check=True)
+    g_recomp = Q.qlora_linear_bwd_ex(q, A, B, r, 2.0 * r, X, None, dY, adapter=ids, p=p,
+                                     keep_mask=md, x_drop=xdrop, check=True)
+    torch.cuda.synchronize()
+    for a, b, name in zip(g_saved, g_recomp, ("dX", "dA", "dB")):
+        assert torch.equal(a, b), name
