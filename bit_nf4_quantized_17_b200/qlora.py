@@ -160,6 +160,29 @@ def qlora_linear_workspace(M, N, K, r):
     return f.value, b.value
 
 
+def _check_linear(q, M, rt, **tensors):
+    """The library sees only pointers: check each tensor's shape, dtype, device and
+    layout here, so that a mismatch raises instead of reading or writing past a buffer.
+    Names: A, B, X, Y, U, dY, dX, dA, dB, adapter, keep_mask, x_drop (None = absent)."""
+    K, N = q.cols, q.rows
+    spec = {
+        "A": ((rt, K), torch.bfloat16), "B": ((N, rt), torch.bfloat16),
+        "X": ((M, K), torch.bfloat16), "Y": ((M, N), torch.bfloat16),
+        "U": ((M, rt), torch.float32), "dY": ((M, N), torch.bfloat16),
+        "dX": ((M, K), torch.bfloat16), "dA": ((rt, K), torch.float32),
+        "dB": ((N, rt), torch.float32), "adapter": ((M,), torch.int32),
+        "keep_mask": ((M, K // 8), torch.uint8), "x_drop": ((M, K), torch.bfloat16),
+    }
+    for name, t in tensors.items():
+        if t is None:
+            continue
+        shape, dtype = spec[name]
+        if tuple(t.shape) != shape or t.dtype != dtype or not t.is_contiguous() or not t.is_cuda:
+            raise ValueError(f"{name}: expected a contiguous CUDA {dtype} tensor of shape "
+                             f"{shape}, got {t.dtype} {tuple(t.shape)} on {t.device}"
+                             f"{'' if t.is_contiguous() else ', not contiguous'}")
+
+
 def _workspace(nbytes, device):
     return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
 
@@ -233,6 +256,7 @@ def qlora_linear_fwd(q, A, B, alpha, X, Y=None, U_save=None, workspace=None, str
     r = A.shape[0]
     if Y is None:
         Y = torch.empty((M, q.rows), dtype=torch.bfloat16, device=X.device)
+    _check_linear(q, M, r, A=A, B=B, X=X, Y=Y, U=U_save)
     if workspace is None:
         workspace = _workspace(qlora_linear_workspace(M, q.rows, q.cols, r)[0], X.device)
     st = q.struct
@@ -253,9 +277,9 @@ def qlora_linear_fwd_multi(q, A, B, r, alpha, adapter, X, Y=None, U_save=None, w
     if rt % r:
         raise ValueError(f"A has {rt} rows: not a stack of rank-{r} adapters")
     n = rt // r
-    assert adapter.dtype == torch.int32 and adapter.numel() == M
     if Y is None:
         Y = torch.empty((M, q.rows), dtype=torch.bfloat16, device=X.device)
+    _check_linear(q, M, rt, A=A, B=B, X=X, Y=Y, U=U_save, adapter=adapter)
     if workspace is None:
         workspace = _workspace(qlora_linear_workspace(M, q.rows, q.cols, rt)[0], X.device)
     st = q.struct
@@ -278,13 +302,14 @@ def qlora_linear_bwd_multi(q, A, B, r, alpha, adapter, X, U, dY, dX=None, dA=Non
         raise ValueError(f"A has {rt} rows: not a stack of rank-{r} adapters")
     n = rt // r
     dev = X.device
-    assert adapter.dtype == torch.int32 and adapter.numel() == M
     if want_dx and dX is None:
         dX = torch.empty((M, q.cols), dtype=torch.bfloat16, device=dev)
     if dA is None:
         dA = torch.empty((rt, q.cols), dtype=torch.float32, device=dev)
     if dB is None:
         dB = torch.empty((q.rows, rt), dtype=torch.float32, device=dev)
+    _check_linear(q, M, rt, A=A, B=B, X=X, U=U, dY=dY, dX=dX if want_dx else None, dA=dA, dB=dB,
+                  adapter=adapter)
     if workspace is None:
         workspace = _workspace(qlora_linear_workspace(M, q.rows, q.cols, rt)[1], dev)
     st = q.struct
@@ -330,6 +355,8 @@ def qlora_linear_fwd_ex(q, A, B, r, alpha, X, adapter=None, p=0.0, keep_mask=Non
     o = _opts(r, A, adapter, p, keep_mask, x_drop)
     if Y is None:
         Y = torch.empty((M, q.rows), dtype=torch.bfloat16, device=X.device)
+    _check_linear(q, M, rt, A=A, B=B, X=X, Y=Y, U=U_save, adapter=adapter, keep_mask=keep_mask,
+                  x_drop=x_drop)
     if workspace is None:
         workspace = _workspace(qlora_linear_workspace(M, q.rows, q.cols, rt)[0], X.device)
     st = q.struct
@@ -356,6 +383,8 @@ def qlora_linear_bwd_ex(q, A, B, r, alpha, X, U, dY, adapter=None, p=0.0, keep_m
         dA = torch.empty((rt, q.cols), dtype=torch.float32, device=dev)
     if dB is None:
         dB = torch.empty((q.rows, rt), dtype=torch.float32, device=dev)
+    _check_linear(q, M, rt, A=A, B=B, X=X, U=U, dY=dY, dX=dX if want_dx else None, dA=dA, dB=dB,
+                  adapter=adapter, keep_mask=keep_mask, x_drop=x_drop)
     if workspace is None:
         workspace = _workspace(qlora_linear_workspace(M, q.rows, q.cols, rt)[1], dev)
     st = q.struct
@@ -382,6 +411,7 @@ def qlora_linear_bwd(q, A, B, alpha, X, U, dY, dX=None, dA=None, dB=None, accumu
         dA = torch.empty((r, q.cols), dtype=torch.float32, device=dev)
     if dB is None:
         dB = torch.empty((q.rows, r), dtype=torch.float32, device=dev)
+    _check_linear(q, M, r, A=A, B=B, X=X, U=U, dY=dY, dX=dX if want_dx else None, dA=dA, dB=dB)
     if workspace is None:
         workspace = _workspace(qlora_linear_workspace(M, q.rows, q.cols, r)[1], dev)
     st = q.struct
@@ -403,6 +433,10 @@ def qlora_merge(q, A, B, alpha, out=None, stream=None):
     r = A.shape[0]
     out = out if out is not None else torch.empty((q.rows, q.cols), dtype=torch.bfloat16,
                                                   device=A.device)
+    _check_linear(q, 0, r, A=A, B=B)
+    if (tuple(out.shape) != (q.rows, q.cols) or out.dtype != torch.bfloat16
+            or not out.is_contiguous()):
+        raise ValueError(f"out: expected a contiguous bf16 tensor of shape {(q.rows, q.cols)}")
     st = q.struct
     _ok(lib().qlora_merge(ctypes.byref(st), _ptr(A), _ptr(B), r, float(alpha), _ptr(out),
                           _stream(stream)), "qlora_merge")
@@ -415,6 +449,10 @@ def qlora_merge_dense(W, A, B, alpha, out=None, stream=None):
     r = A.shape[0]
     rows, cols = W.shape
     out = out if out is not None else torch.empty_like(W)
+    for name, t, shape in (("W", W, (rows, cols)), ("A", A, (r, cols)), ("B", B, (rows, r)),
+                           ("out", out, (rows, cols))):
+        if tuple(t.shape) != shape or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError(f"{name}: expected a contiguous bf16 tensor of shape {shape}")
     _ok(lib().qlora_merge_dense(_ptr(W), rows, cols, _ptr(A), _ptr(B), r, float(alpha), _ptr(out),
                                 _stream(stream)), "qlora_merge_dense")
     return out

@@ -211,3 +211,20 @@ def test_timeout_selftest_argument_errors_without_cuda():
     assert L.qlora_selftest_timeout(0, P(0x10000), None) == Q.QLORA_ERR_SHAPE
     assert L.qlora_selftest_timeout(2 ** 33, P(0x10000), None) == Q.QLORA_ERR_SHAPE
     assert L.qlora_selftest_timeout(1000, P(0x10004), None) == Q.QLORA_ERR_ALIGN
+
+
+def test_binding_checks_tensors_before_calling_the_library():
+    # the library sees only pointers: a wrong shape, dtype or device raises in Python
+    import torch
+    from types import SimpleNamespace
+
+    q = SimpleNamespace(rows=64, cols=128)
+    A = torch.zeros(8, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="A"):
+        Q._check_linear(q, 4, 16, A=A)                       # 8 rows for rank 16
+    with pytest.raises(ValueError, match="keep_mask"):
+        Q._check_linear(q, 4, 8, keep_mask=torch.zeros(4, 8, dtype=torch.uint8))  # K/8 = 16
+    with pytest.raises(ValueError, match="adapter"):
+        Q._check_linear(q, 4, 8, adapter=torch.zeros(4, dtype=torch.int64))
+    with pytest.raises(ValueError, match="cpu"):
+        Q._check_linear(q, 4, 8, A=A)                        # right shape, host memory
