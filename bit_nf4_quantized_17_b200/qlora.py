@@ -228,6 +228,8 @@ def qlora_quantize(W, blocksize=64, dq_blocksize=256, table=QLORA_TABLE_NF4, out
     assert W.is_cuda and W.dim() == 2 and W.is_contiguous() and W.dtype in _DTYPE
     rows, cols = W.shape
     q = out or QuantizedWeight.empty(rows, cols, blocksize, dq_blocksize, table, W.device)
+    if (q.rows, q.cols) != (rows, cols):
+        raise ValueError(f"out holds a {q.rows} x {q.cols} weight, W is {rows} x {cols}")
     if workspace is None:
         workspace = _workspace(qlora_nf4_sizes(rows, cols, blocksize, dq_blocksize)["workspace"],
                                W.device)
@@ -242,6 +244,9 @@ def qlora_quantize(W, blocksize=64, dq_blocksize=256, table=QLORA_TABLE_NF4, out
 def qlora_dequantize(q, dtype=torch.float32, out=None, stream=None):
     out = out if out is not None else torch.empty((q.rows, q.cols), dtype=dtype,
                                                   device=q.codes.device)
+    if tuple(out.shape) != (q.rows, q.cols) or out.dtype not in _DTYPE or not out.is_contiguous():
+        raise ValueError(f"out: expected a contiguous fp32 or bf16 tensor of shape "
+                         f"{(q.rows, q.cols)}")
     st = q.struct
     _ok(lib().qlora_dequantize(ctypes.byref(st), _ptr(out), _DTYPE[out.dtype], _stream(stream)),
         "qlora_dequantize")

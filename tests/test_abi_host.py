@@ -228,3 +228,24 @@ def test_binding_checks_tensors_before_calling_the_library():
         Q._check_linear(q, 4, 8, adapter=torch.zeros(4, dtype=torch.int64))
     with pytest.raises(ValueError, match="cpu"):
         Q._check_linear(q, 4, 8, A=A)                        # right shape, host memory
+
+
+def test_quantize_binding_refuses_a_mismatched_output():
+    # out's dimensions, not W's, would size the library's reads: they must agree
+    import torch
+
+    class FakeW:  # passes the binding's first checks without a GPU
+        is_cuda = True
+        shape = (64, 128)
+        dtype = torch.bfloat16
+
+        def dim(self):
+            return 2
+
+        def is_contiguous(self):
+            return True
+
+    from types import SimpleNamespace
+    out = SimpleNamespace(rows=64, cols=256)
+    with pytest.raises(ValueError, match="64 x 256"):
+        Q.qlora_quantize(FakeW(), out=out)
