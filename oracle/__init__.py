@@ -58,7 +58,7 @@ from .nf4 import (
     compute_weight,
     storage_bits,
 )
-from .linear import lora_scale, linear_fwd, linear_bwd, merge_weight
+from .linear import lora_scale, linear_fwd, linear_bwd, lora_down, lora_grads, merge_weight
 from .optim import adamw_step
 from .multi import linear_fwd_multi, linear_bwd_multi
 from .dropout import unpack_keep_mask, linear_fwd_dropout, linear_bwd_dropout
@@ -68,7 +68,7 @@ __all__ = [
     "nf4_levels", "nf4_raw_quantiles", "uniform_levels", "nearest_level",
     "block_absmax", "pack_nibbles", "unpack_nibbles", "fixed_point_mean",
     "double_quantize", "dequantize_scales", "block_scales", "quantize", "dequantize", "compute_weight",
-    "storage_bits", "lora_scale", "linear_fwd", "linear_bwd", "merge_weight", "adamw_step",
+    "storage_bits", "lora_scale", "linear_fwd", "linear_bwd", "lora_down", "lora_grads", "merge_weight", "adamw_step",
     "linear_fwd_multi", "linear_bwd_multi", "unpack_keep_mask", "linear_fwd_dropout",
     "linear_bwd_dropout",
 ]

@@ -36,13 +36,30 @@ def _f64(a):
     return np.asarray(a).astype(F64)
 
 
+def lora_down(a, x):
+    """U = X A^T in fp64: the LoRA branch's first product A x for every token
+    row (the pages' A x, with tokens as rows)."""
+    return _f64(x) @ _f64(a).T
+
+
 def linear_fwd(w_hat, a, b, alpha, x):
     """Returns (Y, U) in fp64: U = X A^T, Y = X W^T + s U B^T."""
     w, a, b, x = _f64(w_hat), _f64(a), _f64(b), _f64(x)
     s = lora_scale(alpha, a.shape[0])
-    u = x @ a.T
+    u = lora_down(a, x)
     y = x @ w.T + s * (u @ b.T)
     return y, u
+
+
+def lora_grads(a, b, alpha, x, dy):
+    """Returns (dA, dB) in fp64: the adapters' gradients of the backward pass,
+    V = dY B, dB = s dY^T (X A^T), dA = s V^T X.  They need no W; every
+    token row contributes a term, so they are taken over all rows given."""
+    a, b, x, dy = _f64(a), _f64(b), _f64(x), _f64(dy)
+    s = lora_scale(alpha, a.shape[0])
+    v = dy @ b
+    u = lora_down(a, x)
+    return s * (v.T @ x), s * (dy.T @ u)
 
 
 def linear_bwd(w_hat, a, b, alpha, x, dy):
@@ -50,10 +67,8 @@ def linear_bwd(w_hat, a, b, alpha, x, dy):
     w, a, b, x, dy = _f64(w_hat), _f64(a), _f64(b), _f64(x), _f64(dy)
     s = lora_scale(alpha, a.shape[0])
     v = dy @ b
-    u = x @ a.T
     dx = dy @ w + s * (v @ a)
-    db = s * (dy.T @ u)
-    da = s * (v.T @ x)
+    da, db = lora_grads(a, b, alpha, x, dy)
     return dx, da, db
 
 
