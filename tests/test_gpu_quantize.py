@@ -111,3 +111,50 @@ def test_nonfinite_weight_is_reported():
     with pytest.raises(Q.QloraError) as e:
         Q.qlora_quantize(W.to(DEV))
     assert e.value.status == Q.QLORA_ERR_NONFINITE
+
+
+def _threshold_weights(levels, scales, blocks_per_scale, seed):
+    """fp32 weights whose normalised values x = w / s sit on the decision
+    thresholds of `levels` and on their -3..+3 fp32 neighbours.
+
+    Every block of 64 holds one element +-s (so its absmax is exactly s) and
+    63 values w = m s moved by -3..+3 ulps, m the exact midpoint of two
+    adjacent levels (fp64; the decision boundary of the nearest-level rule).
+    With s = 1 the normalised value is w itself, so the kernel's comparison
+    meets each threshold and its neighbours exactly; other scales put
+    RN(w / s) within a few ulps of the thresholds, where the library's cell
+    lookup hands over to its IEEE-division fallback."""
+    q = np.asarray(levels, np.float32).astype(np.float64)
+    mids = (q[:-1] + q[1:]) * 0.5
+    rng = np.random.default_rng(seed)
+    blocks = []
+    for s in scales:
+        s32 = np.float32(s)
+        vals = []
+        for m in mids:
+            c = np.float32(m * np.float64(s32))
+            for d in range(-3, 4):
+                v = c
+                for _ in range(abs(d)):
+                    v = np.nextafter(v, np.float32(np.inf if d > 0 else -np.inf), dtype=np.float32)
+                vals.append(v)
+        vals = np.array(vals, np.float32)
+        assert np.all(np.abs(vals) < s32)
+        for b in range(blocks_per_scale):
+            pick = rng.permutation(np.resize(rng.permutation(vals), 63))
+            block = np.concatenate([[s32 if b % 2 == 0 else -s32], pick]).astype(np.float32)
+            blocks.append(rng.permutation(block))
+    return np.stack(blocks).reshape(-1, 1024)
+
+
+@pytest.mark.parametrize("table", [Q.QLORA_TABLE_NF4, Q.QLORA_TABLE_UNIFORM])
+@pytest.mark.parametrize("dq", [256, 0])
+def test_values_on_every_decision_threshold(table, dq):
+    # codes must match the oracle bit for bit exactly where the nearest level
+    # changes (ties take the lower index), for unit and non-unit scales
+    levels = oracle.nf4_levels() if table == Q.QLORA_TABLE_NF4 else oracle.uniform_levels()
+    scales = [1.0, 0.5, 2.0, 0.02, 0.0173, 3.7, 1e-3, 0.3, 7.25, 1.5 * 2.0 ** -126, 3e-39]
+    W = torch.from_numpy(_threshold_weights(levels, scales, 32, 21 + table))
+    _, ref = _check(W, 64, dq, table)
+    # the inputs do reach every index on both sides of every threshold
+    assert set(np.unique(ref["idx"]).tolist()) == set(range(16))
