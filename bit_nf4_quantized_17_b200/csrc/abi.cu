@@ -9,14 +9,50 @@
 #include <tuple>
 #include <vector>
 
-#include <nvtx3/nvToolsExt.h>
-
 #include "internal.cuh"
 #include "kernels.cuh"
 #include "linear.cuh"
 #include "tc_ptx.cuh"
 
 using namespace qlora;
+
+namespace qlora {
+
+static constexpr int64_t kMaxElems = int64_t(1) << 36;
+
+static bool pow2_in(int32_t v, int32_t lo, int32_t hi) {
+  return v >= lo && v <= hi && (v & (v - 1)) == 0;
+}
+
+const LevelTable* level_table(int32_t table) {
+  static LevelTable tabs[2];
+  static qlora_status ok[2];
+  static std::once_flag once;
+  std::call_once(once, [] {
+    ok[0] = make_level_table(QLORA_TABLE_NF4, &tabs[0]);
+    ok[1] = make_level_table(QLORA_TABLE_UNIFORM, &tabs[1]);
+  });
+  if (table < 0 || table > 1 || ok[table] != QLORA_OK) return nullptr;
+  return &tabs[table];
+}
+
+qlora_status check_nf4_shape(const qlora_nf4& q) {
+  if (q.rows < 1 || q.cols < 1 || q.rows > kMaxElems / q.cols) return QLORA_ERR_SHAPE;
+  if (!pow2_in(q.blocksize, 64, 1024)) return QLORA_ERR_UNSUPPORTED;
+  if (q.dq_blocksize != 0 && !pow2_in(q.dq_blocksize, 64, 1024)) return QLORA_ERR_UNSUPPORTED;
+  if (q.table != QLORA_TABLE_NF4 && q.table != QLORA_TABLE_UNIFORM) return QLORA_ERR_UNSUPPORTED;
+  return QLORA_OK;
+}
+
+qlora_status check_nf4_ptrs(const qlora_nf4& q) {
+  if (!q.codes || !q.factors) return QLORA_ERR_NULL;
+  if (q.dq_blocksize && (!q.scale_codes || !q.mean)) return QLORA_ERR_NULL;
+  if (!aligned16(q.codes) || !aligned16(q.factors)) return QLORA_ERR_ALIGN;
+  if (q.dq_blocksize && (!aligned16(q.scale_codes) || !aligned16(q.mean))) return QLORA_ERR_ALIGN;
+  return QLORA_OK;
+}
+
+}  // namespace qlora
 
 namespace {
 std::atomic<uint64_t> g_launches{0};
@@ -128,40 +164,6 @@ qlora_status qlora::after_launch(const char* kernel, cudaStream_t s) {
 
 namespace {
 
-constexpr int64_t kMaxElems = int64_t(1) << 36;
-
-bool pow2_in(int32_t v, int32_t lo, int32_t hi) {
-  return v >= lo && v <= hi && (v & (v - 1)) == 0;
-}
-
-const LevelTable* level_table(int32_t table) {
-  static LevelTable tabs[2];
-  static qlora_status ok[2];
-  static std::once_flag once;
-  std::call_once(once, [] {
-    ok[0] = make_level_table(QLORA_TABLE_NF4, &tabs[0]);
-    ok[1] = make_level_table(QLORA_TABLE_UNIFORM, &tabs[1]);
-  });
-  if (table < 0 || table > 1 || ok[table] != QLORA_OK) return nullptr;
-  return &tabs[table];
-}
-
-qlora_status check_nf4_shape(const qlora_nf4& q) {
-  if (q.rows < 1 || q.cols < 1 || q.rows > kMaxElems / q.cols) return QLORA_ERR_SHAPE;
-  if (!pow2_in(q.blocksize, 64, 1024)) return QLORA_ERR_UNSUPPORTED;
-  if (q.dq_blocksize != 0 && !pow2_in(q.dq_blocksize, 64, 1024)) return QLORA_ERR_UNSUPPORTED;
-  if (q.table != QLORA_TABLE_NF4 && q.table != QLORA_TABLE_UNIFORM) return QLORA_ERR_UNSUPPORTED;
-  return QLORA_OK;
-}
-
-qlora_status check_nf4_ptrs(const qlora_nf4& q) {
-  if (!q.codes || !q.factors) return QLORA_ERR_NULL;
-  if (q.dq_blocksize && (!q.scale_codes || !q.mean)) return QLORA_ERR_NULL;
-  if (!aligned16(q.codes) || !aligned16(q.factors)) return QLORA_ERR_ALIGN;
-  if (q.dq_blocksize && (!aligned16(q.scale_codes) || !aligned16(q.mean))) return QLORA_ERR_ALIGN;
-  return QLORA_OK;
-}
-
 size_t quantize_workspace(int64_t n, int32_t bs, int32_t dq) {
   const int64_t nb = ceil_div(n, bs);
   return dq ? 512 + static_cast<size_t>(ceil_div(4 * nb, 256) * 256) : 512;
@@ -170,15 +172,6 @@ size_t quantize_workspace(int64_t n, int32_t bs, int32_t dq) {
 }  // namespace
 
 namespace {
-// An NVTX range around an ABI call, so that profiles show the library's calls
-// (free when no tool is attached).
-struct NvtxRange {
-  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
-  ~NvtxRange() { nvtxRangePop(); }
-  NvtxRange(const NvtxRange&) = delete;
-  NvtxRange& operator=(const NvtxRange&) = delete;
-};
-
 // One CTA waits on an mbarrier that nothing completes, with the library's
 // bounded wait, and reports the timeout the way the real kernels do.
 __global__ void timeout_selftest_kernel(long long limit, DeviceStatus* st) {

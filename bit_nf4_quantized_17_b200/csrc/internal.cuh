@@ -7,6 +7,8 @@
 
 #include "qlora.h"
 
+#include <nvtx3/nvToolsExt.h>
+
 namespace qlora {
 
 // First 256 bytes of every workspace: a status word written by kernels that
@@ -34,6 +36,23 @@ struct LevelTable {
 
 // tables.cpp
 qlora_status make_level_table(int32_t table, LevelTable* out);
+
+// abi.cu: the argument checks every call on a quantised weight shares.
+// check_nf4_shape: sizes, block sizes and table; check_nf4_ptrs: the device
+// arrays present and 16-byte aligned.  level_table: the library's level and
+// threshold table of QLORA_TABLE_NF4 / QLORA_TABLE_UNIFORM (nullptr otherwise).
+qlora_status check_nf4_shape(const qlora_nf4& q);
+qlora_status check_nf4_ptrs(const qlora_nf4& q);
+const LevelTable* level_table(int32_t table);
+
+// An NVTX range around an ABI call, so that profiles show the library's calls
+// (free when no tool is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 

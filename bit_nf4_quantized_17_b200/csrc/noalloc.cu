@@ -12,7 +12,10 @@
 // Limits and sharing:
 //   * the array holds 512 bytes of reduction words plus one fp32 per block,
 //     for at most kMaxBlocks blocks (2^20, i.e. 64 Mi weights at blocksize
-//     64); larger tensors are refused with QLORA_ERR_WORKSPACE;
+//     64); larger double-quantised tensors are refused with
+//     QLORA_ERR_WORKSPACE.  Without double quantisation the block absmax
+//     goes straight to q->factors and only the 512-byte header is used, so
+//     that case has no size limit beyond qlora_quantize's own;
 //   * every GPU that loads the library keeps its own copy of the array
 //     (4 MiB + 512 B) until the process exits;
 //   * all calls on a device share it: two calls whose work overlaps on the
@@ -23,7 +26,6 @@
 // The first call on a device looks up the array's device address with
 // cudaGetSymbolAddress (with that device current); make that first call
 // before any stream capture.
-#include <cstring>
 #include <mutex>
 
 #include "internal.cuh"
@@ -54,10 +56,6 @@ void* scratch_on_current_device() {
   return g_scratch_addr[dev];
 }
 
-bool pow2_between(int32_t v, int32_t lo, int32_t hi) {
-  return v >= lo && v <= hi && (v & (v - 1)) == 0;
-}
-
 }  // namespace
 }  // namespace qlora
 
@@ -65,27 +63,19 @@ extern "C" qlora_status qlora_quantize_noalloc(const void* W, int32_t w_dtype,
                                                const qlora_nf4* q, uint32_t* status_out,
                                                void* stream) {
   using namespace qlora;
+  const NvtxRange nvtx("qlora_quantize_noalloc");
   if (!q || !W) return QLORA_ERR_NULL;
-  if (q->rows < 1 || q->cols < 1 || q->rows > (int64_t(1) << 36) / q->cols) return QLORA_ERR_SHAPE;
-  if (!pow2_between(q->blocksize, 64, 1024)) return QLORA_ERR_UNSUPPORTED;
-  if (q->dq_blocksize != 0 && !pow2_between(q->dq_blocksize, 64, 1024)) return QLORA_ERR_UNSUPPORTED;
+  qlora_status st = check_nf4_shape(*q);
+  if (st != QLORA_OK) return st;
+  if ((st = check_nf4_ptrs(*q)) != QLORA_OK) return st;
   if (w_dtype != QLORA_F32 && w_dtype != QLORA_BF16) return QLORA_ERR_UNSUPPORTED;
-  if (!q->codes || !q->factors || (q->dq_blocksize && (!q->scale_codes || !q->mean)))
-    return QLORA_ERR_NULL;
-  if (!aligned16(W) || !aligned16(q->codes) || !aligned16(q->factors) ||
-      (q->dq_blocksize && (!aligned16(q->scale_codes) || !aligned16(q->mean))) ||
-      (status_out && (reinterpret_cast<uintptr_t>(status_out) & 3u)))
+  if (!aligned16(W) || (status_out && (reinterpret_cast<uintptr_t>(status_out) & 3u)))
     return QLORA_ERR_ALIGN;
-  if (ceil_div(q->rows * q->cols, q->blocksize) > kMaxBlocks) return QLORA_ERR_WORKSPACE;
-
-  static LevelTable tables[2];
-  static qlora_status table_ok[2];
-  static std::once_flag once;
-  std::call_once(once, [] {
-    table_ok[0] = make_level_table(QLORA_TABLE_NF4, &tables[0]);
-    table_ok[1] = make_level_table(QLORA_TABLE_UNIFORM, &tables[1]);
-  });
-  if (q->table < 0 || q->table > 1 || table_ok[q->table] != QLORA_OK) return QLORA_ERR_UNSUPPORTED;
+  // the per-block absmax lives in the array only with double quantisation
+  if (q->dq_blocksize != 0 && ceil_div(q->rows * q->cols, q->blocksize) > kMaxBlocks)
+    return QLORA_ERR_WORKSPACE;
+  const LevelTable* table = level_table(q->table);
+  if (!table) return QLORA_ERR_UNSUPPORTED;
 
   void* scratch = scratch_on_current_device();
   if (!scratch) return QLORA_ERR_CUDA;
@@ -93,7 +83,7 @@ extern "C" qlora_status qlora_quantize_noalloc(const void* W, int32_t w_dtype,
   // the array keeps the previous call's contents: clear the status word and
   // the reduction words (the quantiser clears the latter again itself)
   if (cudaMemsetAsync(scratch, 0, kHeaderBytes, s) != cudaSuccess) return QLORA_ERR_CUDA;
-  qlora_status st = launch_quantize(W, w_dtype, *q, tables[q->table], scratch, s);
+  st = launch_quantize(W, w_dtype, *q, *table, scratch, s);
   if (st != QLORA_OK) return st;
   if (status_out &&
       cudaMemcpyAsync(status_out, scratch, sizeof(uint32_t), cudaMemcpyDeviceToDevice, s) !=

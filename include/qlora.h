@@ -131,10 +131,16 @@ qlora_status qlora_quantize(const void* W, int32_t w_dtype, const qlora_nf4* q,
  * of cudaMalloc/cudaFree.  The pages have no counterpart to this call; it is a
  * library convenience.  Same inputs, outputs and results as qlora_quantize.
  * The reduction workspace is a fixed array in the library's own device memory
- * (one copy per GPU that loads the library, 4 MiB + 512 B, kept until exit):
- * at most 2^20 blocks (64 Mi weights at blocksize 64), larger tensors return
- * QLORA_ERR_WORKSPACE.  All calls on a device share the array: calls whose
- * work overlaps on the GPU race; calls on one stream are safe.  status_out
+ * (one copy per GPU that loads the library, 4 MiB + 512 B, kept until exit).
+ * With double quantisation it holds one fp32 per block: at most 2^20 blocks
+ * (64 Mi weights at blocksize 64), larger tensors return QLORA_ERR_WORKSPACE
+ * before any work is enqueued.  Without double quantisation (dq_blocksize 0)
+ * only its 512-byte header is used and there is no such limit.  Argument
+ * checks and their errors are those of qlora_quantize.  All calls on a
+ * device share the array: calls whose work overlaps on the GPU race; calls on
+ * one stream are safe.  Each call clears the words that must start at zero
+ * (status, maximum, sum) and rewrites the per-block values before reading
+ * them, so nothing carries over from an earlier call.  status_out
  * (device, 4 bytes, may be NULL) receives the device status when the work
  * completes: 0, or QLORA_ERR_NONFINITE for a NaN or infinite weight.  The
  * first call on a device looks up the array (cudaGetSymbolAddress on the

@@ -29,9 +29,9 @@ def _noalloc_fn():
     return fn
 
 
-def _quantize_noalloc(W, blocksize, dq_blocksize):
-    q = Q.QuantizedWeight.empty(W.shape[0], W.shape[1], blocksize, dq_blocksize,
-                                Q.QLORA_TABLE_NF4, W.device)
+def _quantize_noalloc(W, blocksize, dq_blocksize, table=Q.QLORA_TABLE_NF4):
+    q = Q.QuantizedWeight.empty(W.shape[0], W.shape[1], blocksize, dq_blocksize, table,
+                                W.device)
     status = torch.full((1,), 12345, dtype=torch.int32, device=W.device)
     st = q.struct
     dtype = Q.QLORA_BF16 if W.dtype == torch.bfloat16 else Q.QLORA_F32
@@ -67,3 +67,32 @@ def test_noalloc_quantize_refuses_tensors_beyond_its_array():
     big = Q.qlora_nf4(1 << 20, 65, 64, 256, 0, 0, 0x10000, 0x20000, 0x30000, 0x40000)
     rc = _noalloc_fn()(ctypes.c_void_p(0x50000), Q.QLORA_BF16, ctypes.byref(big), None, None)
     assert rc == Q.QLORA_ERR_WORKSPACE
+
+
+def test_noalloc_quantize_at_the_array_limit_and_without_double_quant():
+    # exactly 2^20 blocks with double quantisation is accepted; without it
+    # only the header of the array is used, so a larger tensor is accepted too
+    dev = torch.device("cuda")
+    W = WL.randn((1024, 65536), 0.02, 91, torch.bfloat16, dev)        # 2^20 blocks of 64
+    got, status = _quantize_noalloc(W, 64, 256)
+    assert status == 0
+    _same(got, Q.qlora_quantize(W, 64, 256))
+    W2 = WL.randn((1025, 65536), 0.02, 92, torch.bfloat16, dev)       # 2^20 + 1024 blocks
+    for table in (Q.QLORA_TABLE_NF4, Q.QLORA_TABLE_UNIFORM):
+        got, status = _quantize_noalloc(W2, 64, 0, table)
+        assert status == 0
+        _same(got, Q.qlora_quantize(W2, 64, 0, table))
+
+
+def test_noalloc_nonfinite_status_does_not_carry_over():
+    # a NaN weight reports QLORA_ERR_NONFINITE through status_out; the next
+    # call on a clean weight reports 0 and equals qlora_quantize bit for bit
+    dev = torch.device("cuda")
+    W = WL.randn((512, 1024), 0.02, 93, torch.float32, dev)
+    bad = W.clone()
+    bad[17, 300] = float("nan")
+    _, status = _quantize_noalloc(bad, 64, 256)
+    assert status == Q.QLORA_ERR_NONFINITE
+    got, status = _quantize_noalloc(W, 64, 256)
+    assert status == 0
+    _same(got, Q.qlora_quantize(W, 64, 256))
