@@ -89,6 +89,99 @@ def test_gradient_allreduce_equals_full_batch(world):
     assert np.array_equal(got[0][0], got[1][0]) and np.array_equal(got[0][1], got[1][1])
 
 
+# a small stack: 3 layers x 3 linears of different shapes (r, d_in, d_out)
+STACK = [(4, 128, 24), (4, 64, 128), (8, 128, 64)]
+LAYERS = 3
+M_STACK = 13
+
+
+def _stack_problem():
+    rng = np.random.default_rng(11)
+    layers = []
+    for _ in range(LAYERS):
+        row = []
+        for r, k, n in STACK:
+            w = (rng.standard_normal((n, k)) * 0.02).astype(np.float32)
+            w_hat = oracle.compute_weight(oracle.quantize(w, 64, 256)).reshape(n, k)
+            row.append((w_hat, rng.standard_normal((r, k)) / np.sqrt(r),
+                        rng.standard_normal((n, r)) * 0.05, rng.standard_normal((M_STACK, k)),
+                        rng.standard_normal((M_STACK, n))))
+        layers.append(row)
+    return layers
+
+
+def _stack_rank_main(rank, world, port, queue):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        layers = _stack_problem()
+        lo, hi = dp.token_shard(M_STACK, rank, world)
+        buckets = [dp.LayerBucket(STACK, "cpu") for _ in range(LAYERS)]
+        works = []
+        # the bench's order: backward from the last layer down, each layer's
+        # exchange started as soon as its gradients are written
+        for l in reversed(range(LAYERS)):
+            for j in reversed(range(len(STACK))):
+                w_hat, a, b, x, dy = layers[l][j]
+                _, da, db = oracle.linear_bwd(w_hat, a, b, ALPHA, x[lo:hi], dy[lo:hi])
+                dA, dB = buckets[l].views[j]
+                dA.copy_(torch.from_numpy(np.asarray(da, np.float32)))
+                dB.copy_(torch.from_numpy(np.asarray(db, np.float32)))
+            works.append(buckets[l].allreduce(async_op=True))
+        for wk in works:
+            wk.wait()
+        queue.put((rank, [[(v[0].double().numpy(), v[1].double().numpy()) for v in bk.views]
+                          for bk in buckets]))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_layer_buckets_exchanged_per_layer_equal_full_batch():
+    world = 2
+    ctx = mp.get_context("spawn")
+    queue = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_stack_rank_main, args=(r, world, port, queue))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    got = {}
+    for _ in range(world):
+        rank, res = queue.get(timeout=120)
+        got[rank] = res
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    layers = _stack_problem()
+    for l in range(LAYERS):
+        for j in range(len(STACK)):
+            w_hat, a, b, x, dy = layers[l][j]
+            _, da_ref, db_ref = oracle.linear_bwd(w_hat, a, b, ALPHA, x, dy)
+            for rank in range(world):
+                da, db = got[rank][l][j]
+                np.testing.assert_allclose(da, da_ref, rtol=1e-5, atol=1e-6 * np.abs(da_ref).max())
+                np.testing.assert_allclose(db, db_ref, rtol=1e-5, atol=1e-6 * np.abs(db_ref).max())
+            assert np.array_equal(got[0][l][j][0], got[1][l][j][0])
+
+
+def test_layer_bucket_layout():
+    bk = dp.LayerBucket(STACK + [(64, 8192, 22016)], "cpu")
+    base = bk.flat.data_ptr()
+    ends = []
+    for (r, k, n), (dA, dB) in zip(STACK + [(64, 8192, 22016)], bk.views):
+        assert dA.shape == (r, k) and dB.shape == (n, r)
+        assert dA.is_contiguous() and dB.is_contiguous()
+        for v in (dA, dB):
+            assert (v.data_ptr() - base) % 256 == 0
+            ends.append((v.data_ptr() - base, v.data_ptr() - base + 4 * v.numel()))
+    ends.sort()
+    for (a0, a1), (b0, b1) in zip(ends, ends[1:]):
+        assert a1 <= b0  # disjoint, in order
+    assert ends[-1][1] <= 4 * bk.flat.numel()
+    # one rank: no collective, nothing to wait for
+    assert bk.allreduce(async_op=True) is None
+
+
 @pytest.mark.parametrize("total,world", [(4096, 2), (11, 2), (11, 4), (3, 8), (0, 2), (8192, 8)])
 def test_token_shards_partition_the_batch(total, world):
     spans = [dp.token_shard(total, r, world) for r in range(world)]
