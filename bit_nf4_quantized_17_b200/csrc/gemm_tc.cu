@@ -408,33 +408,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 }
 
 // Deterministic split-K reduction.  v = sum_z part[z][i][j] (+ part[z][i][j + lo]
-// when lo > 0), summed in a fixed order; then up to three outputs:
-//   o1  fp32  a1 * v, at [i][j] or transposed [j][i], optionally added to o1
-//   o2  bf16  hi = bf16(a2 v) at [i][j] and, if o2_lo > 0, lo = bf16(a2 v - hi) at [i][j + o2_lo]
-//   o3  bf16  the same pair transposed: hi at [j][i], lo at [j + o3_lo][i]
-// hi + lo carries a2 v to about 16 significant bits through bf16 tensor-core operands.
-__device__ __forceinline__ void reduce_store(float v, int64_t i, int j, float* o1, int64_t ld1,
-                                             int trans1, float a1, int acc1, __nv_bfloat16* o2,
-                                             int64_t ld2, float a2, int o2_lo, __nv_bfloat16* o3,
-                                             int64_t ld3, float a3, int o3_lo) {
-  if (o1) {
-    float* dst = trans1 ? o1 + j * ld1 + i : o1 + i * ld1 + j;
-    *dst = acc1 ? *dst + a1 * v : a1 * v;
-  }
-  if (o2) {
-    const float x = a2 * v;
-    const __nv_bfloat16 h = __float2bfloat16_rn(x);
-    o2[i * ld2 + j] = h;
-    if (o2_lo) o2[i * ld2 + j + o2_lo] = __float2bfloat16_rn(x - __bfloat162float(h));
-  }
-  if (o3) {
-    const float x = a3 * v;
-    const __nv_bfloat16 h = __float2bfloat16_rn(x);
-    o3[j * ld3 + i] = h;
-    if (o3_lo) o3[(j + o3_lo) * ld3 + i] = __float2bfloat16_rn(x - __bfloat162float(h));
-  }
-}
-
+// when lo > 0), summed in a fixed order; then the outputs of tc::reduce_store.
 // With o2_pad the padding columns of o2 ([cols, o2_lo) and [o2_lo + cols,
 // 2 o2_lo) of every row) are written as zeros too, so o2 needs no memset.
 __global__ void splitk_reduce_kernel(const float* __restrict__ part, int splits, int64_t rows,
@@ -477,7 +451,7 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ part, int splits,
       }
     }
     if (seg && __ldg(seg + i) != j / seg_cols) v = 0.0f;
-    reduce_store(v, i, j, o1, ld1, trans1, a1, acc1, o2, ld2, a2, o2_lo, o3, ld3, a3, o3_lo);
+    tc::reduce_store(v, i, j, o1, ld1, trans1, a1, acc1, o2, ld2, a2, o2_lo, o3, ld3, a3, o3_lo);
   }
 }
 
@@ -517,7 +491,7 @@ __global__ void splitk_reduce_warp_kernel(const float* __restrict__ part, int sp
     for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
     if (seg && __ldg(seg + i) != j / seg_cols) v = 0.0f;
     if (lane == 0)
-      reduce_store(v, i, j, o1, ld1, trans1, a1, acc1, o2, ld2, a2, o2_lo, o3, ld3, a3, o3_lo);
+      tc::reduce_store(v, i, j, o1, ld1, trans1, a1, acc1, o2, ld2, a2, o2_lo, o3, ld3, a3, o3_lo);
   }
 }
 

@@ -4,11 +4,13 @@
 // (forward) or dX = dY W + sV A (backward), the 4-bit W dequantised on load
 // to bf16 ("QLoRA技术从入门到精通", 3(2): restore a block to BF16, multiply,
 // discard), the LoRA term added as extra K stages of the same accumulators.
-// Here two CTAs of a cluster compute a 512 x 256 output tile with pair MMAs
-// (tcgen05.mma.cta_group::2, M = 256, N = 256, issued by the even CTA):
+// Here two CTAs of a cluster compute a 512 x tn output tile with pair MMAs
+// (tcgen05.mma.cta_group::2, M = 256, N = tn, issued by the even CTA; tn =
+// 256 for the backward, 192..256 for the forward, chosen per launch so that
+// the tiles fill the last round of pair slots):
 //
 //   * each CTA holds its own 256 activation rows (two 128-row sub-tiles) and
-//     HALF of the B tile: 128 of the 256 W rows (forward) or 128 of the 256
+//     HALF of the B tile: tn / 2 of the W rows (forward) or 128 of the 256
 //     output columns (backward) - the MMA reads the other half from the peer;
 //   * so each SM dequantises half of the W tile per k-tile and its shared
 //     memory carries half of the B traffic, for the same MMA work per SM as
@@ -54,6 +56,8 @@ struct Tc2Args {
   int32_t k2_tiles, k2_half, k2_last_steps;
   int32_t b2_mn;             // extension B operand MN-major (backward)
   int32_t a_bytes;           // bytes of one CTA's activation tile per stage
+  int32_t tn;                // output columns of a pair tile (a multiple of 16, <= 256);
+                             // each CTA holds tn / 2 rows of the B tile
   QView w;
   int32_t kblocks;           // W.cols / 64
   int64_t nblocks;           // entries of w.scale_codes
@@ -106,8 +110,11 @@ tc2_fused_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = ptx::cluster_ctarank();
   const int m0 = static_cast<int>(blockIdx.x >> 1) * 512 + static_cast<int>(rank) * 256;
-  const int n0 = blockIdx.y * 256;                          // output columns of the pair tile
-  const int nh = n0 + static_cast<int>(rank) * 128;         // this CTA's half of B
+  const int hn = p.tn >> 1;                                 // B rows this CTA holds
+  const int n0 = blockIdx.y * p.tn;                         // output columns of the pair tile
+  const int nh = n0 + static_cast<int>(rank) * hn;          // this CTA's half of B
+  const uint32_t code_bytes = (BMODE == B_DQ_K) ? static_cast<uint32_t>(hn) * 32u : kCodeSlot;
+  const uint32_t b_bytes = static_cast<uint32_t>(hn) * 128u;
   const int total = p.kt_total + p.k2_tiles;
 
   if (threadIdx.x == 0) {
@@ -151,7 +158,7 @@ tc2_fused_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           break;
         }
         uint8_t* dst = codes_ring + cs * kCodeSlot;
-        ptx::mbar_arrive_expect_tx(&codes_full[cs], kCodeSlot);
+        ptx::mbar_arrive_expect_tx(&codes_full[cs], code_bytes);
         if (BMODE == B_DQ_K)
           ptx::tma_load_2d(&tmB, &codes_full[cs], dst, kc * 32, nh);  // 128 W rows x 32 bytes
         else
@@ -177,7 +184,7 @@ tc2_fused_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         const int tt = kt - p.kt_total;
         const int k2a = tt * 64;
         const int k2b = (tt % p.k2_half) * 64;
-        if (rank == 0) ptx::mbar_arrive_expect_tx(&full_a[s], 2 * (p.a_bytes + kBBytes));
+        if (rank == 0) ptx::mbar_arrive_expect_tx(&full_a[s], 2 * (p.a_bytes + b_bytes));
         ptx::tma_load_2d_pair(&tmA2, bar, sa, k2a, m0);
         if (p.b2_mn) {
           ptx::tma_load_2d_pair(&tmB2, bar, sb, nh, k2b);
@@ -198,8 +205,8 @@ tc2_fused_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         ptx::mbar_wait_cluster(&full_a[kt % kStages], (kt / kStages) & 1, kTimeoutCycles, nullptr);
   } else if (warp == 1 && lane == 0 && rank == 0) {
     // ------------------------------------------------------ MMA issuer (even CTA)
-    const uint32_t idesc = ptx::idesc_bf16(256, 256, 0, BMODE == B_DQ_MN ? 1 : 0);
-    const uint32_t idesc2 = ptx::idesc_bf16(256, 256, 0, p.b2_mn);
+    const uint32_t idesc = ptx::idesc_bf16(256, p.tn, 0, BMODE == B_DQ_MN ? 1 : 0);
+    const uint32_t idesc2 = ptx::idesc_bf16(256, p.tn, 0, p.b2_mn);
     int done = 0;
     for (int kt = 0; kt < total; ++kt) {
       const int s = kt % kStages;
@@ -241,13 +248,16 @@ tc2_fused_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     const float mu = (p.w.dq_shift >= 0) ? __ldg(p.w.mean) : 0.0f;
     const int row = (BMODE == B_DQ_K) ? td : (td & 63);
     const int q = (BMODE == B_DQ_K) ? 0 : (td >> 6);
+    // forward: the threads past this CTA's hn W rows expand nothing but keep
+    // their barrier arrivals
+    const bool active = (BMODE == B_DQ_K) ? (td < hn) : true;
     const uint32_t leader_full_b0 = ptx::cluster_addr(&full_b[0], 0);
     struct RawScale {
       float q, f;
       bool in;
     };
     auto load_scale = [&](int kt) -> RawScale {
-      if (kt >= p.kt_total) return RawScale{0.0f, 0.0f, false};
+      if (kt >= p.kt_total || !active) return RawScale{0.0f, 0.0f, false};
       const int64_t wrow = (BMODE == B_DQ_K) ? static_cast<int64_t>(nh) + row
                                              : static_cast<int64_t>(kt) * 64 + row;
       const int64_t kb = (BMODE == B_DQ_K) ? kt : (nh / 64 + q);
@@ -271,10 +281,12 @@ tc2_fused_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       r1 = load_scale(kt + 8);
       if (!ptx::mbar_wait(&codes_full[s], ph, kTimeoutCycles, abort_flag)) break;
       const uint8_t* slot = codes_ring + s * kCodeSlot;
-      uint4 c0, c1;
+      uint4 c0 = make_uint4(0u, 0u, 0u, 0u), c1 = c0;
       if (BMODE == B_DQ_K) {
-        c0 = *reinterpret_cast<const uint4*>(slot + row * 32);
-        c1 = *reinterpret_cast<const uint4*>(slot + row * 32 + 16);
+        if (active) {
+          c0 = *reinterpret_cast<const uint4*>(slot + row * 32);
+          c1 = *reinterpret_cast<const uint4*>(slot + row * 32 + 16);
+        }
       } else {
         c0 = *reinterpret_cast<const uint4*>(slot + row * 64 + q * 32);
         c1 = *reinterpret_cast<const uint4*>(slot + row * 64 + q * 32 + 16);
@@ -290,9 +302,11 @@ tc2_fused_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       if (!ptx::mbar_wait(&empty[s], ph ^ 1, kTimeoutCycles, abort_flag)) break;
       uint8_t* sb = smem + s * kStageBytes + kABytes;
       uint8_t* dst_row = (BMODE == B_DQ_K) ? sb + row * 128 : sb + q * 8192 + row * 128;
+      if (active) {
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-        *reinterpret_cast<uint4*>(dst_row + 16 * (j ^ (row & 7))) = expand8(words[j], L, H);
+        for (int j = 0; j < 8; ++j)
+          *reinterpret_cast<uint4*>(dst_row + 16 * (j ^ (row & 7))) = expand8(words[j], L, H);
+      }
       // make the writes visible to the MMA (async proxy, possibly issued by
       // the peer CTA), then one arrival per warp on the even CTA's barrier
       ptx::fence_proxy_async_smem();
@@ -308,7 +322,10 @@ tc2_fused_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       const int cg = (warp - 4) >> 2;  // 0..3: accumulator cg & 1, column half cg >> 1
       const int t = cg & 1;
       const int64_t grow = static_cast<int64_t>(m0) + 128 * t + 32 * quarter + lane;
-      for (int c = (cg >> 1) * 8; c < (cg >> 1) * 8 + 8; ++c) {
+      const int chunks = p.tn >> 4;                 // 16-column chunks of the tile
+      const int c_half = (chunks + 1) >> 1;
+      const int c_begin = (cg >> 1) ? c_half : 0, c_end = (cg >> 1) ? chunks : c_half;
+      for (int c = c_begin; c < c_end; ++c) {
         uint32_t r[16];
         ptx::tmem_ld_x16(tmem + (static_cast<uint32_t>(32 * quarter) << 16) + t * 256 + c * 16, r);
         ptx::tmem_ld_wait();
@@ -365,6 +382,7 @@ Tc2Args args_of(const QView& w, int64_t M, int64_t n_out, int32_t r, void* out, 
   p.k2_tiles = 2 * p.k2_half;
   p.k2_last_steps = ((r - 64 * (p.k2_half - 1)) + 15) / 16;
   p.a_bytes = kABytes;
+  p.tn = 256;
   p.w = w;
   p.kblocks = static_cast<int32_t>(w.cols / 64);
   p.nblocks = (w.rows * w.cols / 64) >> w.bs_shift;
@@ -379,20 +397,49 @@ Tc2Args args_of(const QView& w, int64_t M, int64_t n_out, int32_t r, void* out, 
 
 bool tc2_eligible(int64_t M, const FusedShape& f) { return f.mt == 2 && f.splits == 1 && M > 256; }
 
+// Output columns of a forward pair tile: 256 unless a narrower tile (down to
+// 192, in steps of 16) ends the launch sooner.  An output 8192 wide at 2048
+// tokens is 128 tiles of 256 on 74 pair slots (1.73 waves, two rounds); at
+// 224 it is 148 tiles, two full rounds of narrower tiles.
+static int tc2_pair_tile_width(int64_t M, int64_t n_out) {
+  // pair slots of the device: one CTA per SM (shared memory), two per pair
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    (void)cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t slots = sms >= 2 ? sms / 2 : 1;
+  const int64_t m_pairs = ceil_div(M, 512);
+  // a pair tile's time grows with its width; pick the width that ends the
+  // launch soonest (waves x width), the widest among equals
+  int best = 256;
+  int64_t best_cost = -1;
+  for (int tn = 256; tn >= 192; tn -= 16) {
+    const int64_t tiles = m_pairs * ceil_div(n_out, tn);
+    const int64_t cost = ceil_div(tiles, slots) * tn;
+    if (best_cost < 0 || cost < best_cost) {
+      best = tn;
+      best_cost = cost;
+    }
+  }
+  return best;
+}
+
 qlora_status tc2_fused_forward(const QView& w, const LevelTable& t, const void* X, int64_t M,
                                const void* sU, const void* B, int32_t r, void* Y,
                                DeviceStatus* st, cudaStream_t s) {
   const int64_t N = w.rows, K = w.cols;
+  const int tn = tc2_pair_tile_width(M, N);
+  const uint32_t hn = static_cast<uint32_t>(tn / 2);
   CUtensorMap ma, mb, ma2, mb2;
   if (!make_map(&ma, X, true, K, M, K, 64, 256, true) ||
-      !make_map(&mb, w.codes, false, K / 2, N, K / 2, 32, 128, false) ||
+      !make_map(&mb, w.codes, false, K / 2, N, K / 2, 32, hn, false) ||
       !make_map(&ma2, sU, true, 2 * lora_span(r), M, 2 * lora_span(r), 64, 256, true) ||
-      !make_map(&mb2, B, true, r, N, r, 64, 128, true))
+      !make_map(&mb2, B, true, r, N, r, 64, hn, true))
     return QLORA_ERR_CUDA;
   Tc2Args p = args_of(w, M, N, r, Y, st);
   p.kt_total = static_cast<int32_t>(K / 64);
   p.b2_mn = 0;
-  return launch_tc2<B_DQ_K>(ma, mb, ma2, mb2, p, t, ceil_div(M, 512), ceil_div(N, 256), s);
+  p.tn = tn;
+  return launch_tc2<B_DQ_K>(ma, mb, ma2, mb2, p, t, ceil_div(M, 512), ceil_div(N, tn), s);
 }
 
 qlora_status tc2_fused_dgrad(const QView& w, const LevelTable& t, const void* dY, int64_t M,

@@ -92,6 +92,20 @@ qlora_status tc_lora_gemm(const void* A, bool a_mn, int64_t m_rows, int64_t kdim
                           const void* B, int64_t ld_b, int32_t b_rows, int32_t n_cols,
                           float* part, int splits, DeviceStatus* st, cudaStream_t s);
 
+struct ReduceArgs;
+// gemm_rank.cu: the same product as tc_lora_gemm followed by splitk_reduce,
+// in one launch: the contraction split over the CTAs of a cluster, the fp32
+// partials summed in distributed shared memory in split order, the sums
+// written to the outputs of `out` (its part, splits and pcols are ignored;
+// cols and lo index the n_cols partial columns).  n_cols a multiple of 16 in
+// [16, 256], cols and lo multiples of 4 with cols + lo <= n_cols
+// (tc_rank_eligible); otherwise QLORA_ERR_UNSUPPORTED.
+bool tc_rank_eligible(int32_t n_cols, int32_t cols, int32_t lo);
+int tc_rank_splits(int64_t m_tiles, int64_t k_tiles);
+qlora_status tc_rank_gemm(const void* A, bool a_mn, int64_t m_rows, int64_t kdim, int64_t ld_a,
+                          const void* B, int64_t ld_b, int32_t b_rows, int32_t n_cols,
+                          const ReduceArgs& out, DeviceStatus* st, cudaStream_t s);
+
 struct ReduceArgs {
   const float* part;
   int splits;

@@ -152,6 +152,25 @@ ReduceArgs reduce_args(const float* part, int splits, int64_t rows, int cols, in
   return a;
 }
 
+// A rank-r product and its outputs: one cluster-reduced launch where the
+// partial tile fits (n_cols <= 256), else the split-K GEMM into `part` and
+// the reduction launch.
+qlora_status rank_product(const void* A, bool a_mn, int64_t m_rows, int64_t kdim, int64_t ld_a,
+                          const void* B, int64_t ld_b, int32_t b_rows, int32_t n_cols,
+                          float* part, int splits, const ReduceArgs& out, DeviceStatus* st,
+                          cudaStream_t s) {
+  if (tc_rank_eligible(n_cols, out.cols, out.lo))
+    return tc_rank_gemm(A, a_mn, m_rows, kdim, ld_a, B, ld_b, b_rows, n_cols, out, st, s);
+  qlora_status e = tc_lora_gemm(A, a_mn, m_rows, kdim, ld_a, B, ld_b, b_rows, n_cols, part,
+                                splits, st, s);
+  if (e != QLORA_OK) return e;
+  ReduceArgs ra = out;
+  ra.part = part;
+  ra.splits = splits;
+  ra.pcols = n_cols;
+  return splitk_reduce(ra, s);
+}
+
 }  // namespace
 
 LinearPlan plan_linear(int64_t M, int64_t N, int64_t K, int32_t r) {
@@ -221,7 +240,6 @@ qlora_status linear_forward(const qlora_nf4& W, const LevelTable& t, const void*
     char* su = ws + L.su;
     float* part = reinterpret_cast<float*>(ws + L.part_f);
     // U = X A^T (split-K over d_in) -> U_save (fp32) and sU = s U as bf16 hi + lo
-    QLORA_TRY(tc_lora_gemm(xl, false, M, K, K, A, K, r, r16, part, sp.u, st, s));
     ReduceArgs ra = reduce_args(part, sp.u, M, r, r16);
     ra.seg = seg;  // U / V: each token keeps only its adapter's columns
     ra.seg_cols = r_adapter;
@@ -233,7 +251,7 @@ qlora_status linear_forward(const qlora_nf4& W, const LevelTable& t, const void*
     ra.a2 = sc * o.keep;
     ra.o2_lo = span;
     ra.o2_pad = 1;  // the padding columns meet zero B columns in the MMA: written as zeros
-    QLORA_TRY(splitk_reduce(ra, s));
+    QLORA_TRY(rank_product(xl, false, M, K, K, A, K, r, r16, part, sp.u, ra, st, s));
     // Y = X W^T + sU B^T in one kernel (split over d_in, then summed, when the
     // output alone would leave SMs idle)
     const FusedShape f = fused_shape(M, N, K / 64);
@@ -338,7 +356,6 @@ qlora_status linear_backward(const qlora_nf4& W, const LevelTable& t, const void
     // B^T (r x N) so that V = dY B contracts two K-major operands
     QLORA_TRY(transpose_to_bf16(B, false, N, r, r, bt, N, 0, s));
     // V = dY B -> sV = s V as [hi | lo] and V^T as [hi ; lo]
-    QLORA_TRY(tc_lora_gemm(dY, false, M, N, N, bt, N, r, r16, part, sp.v, st, s));
     {
       ReduceArgs ra = reduce_args(part, sp.v, M, r, r16);
       ra.seg = seg;  // U / V: each token keeps only its adapter's columns
@@ -357,7 +374,7 @@ qlora_status linear_backward(const qlora_nf4& W, const LevelTable& t, const void
       ra.ld3 = mp;
       ra.a3 = 1.0f;
       ra.o3_lo = r16;
-      QLORA_TRY(splitk_reduce(ra, s));
+      QLORA_TRY(rank_product(dY, false, M, N, N, bt, N, r, r16, part, sp.v, ra, st, s));
     }
     // dB and dA on the side stream, dX on the caller's: they share only
     // inputs, and the side stream reuses `part` after V's reduction
@@ -372,7 +389,6 @@ qlora_status linear_backward(const qlora_nf4& W, const LevelTable& t, const void
       if (U) {
         QLORA_TRY(transpose_to_bf16(U, true, M, r, r, ut, mp, r16, s2));
       } else {
-        QLORA_TRY(tc_lora_gemm(xl, false, M, K, K, A, K, r, r16, part, sp.u, st, s2));
         ReduceArgs ra = reduce_args(part, sp.u, M, r, r16);
         ra.seg = seg;  // U / V: each token keeps only its adapter's columns
         ra.seg_cols = r_adapter;
@@ -380,10 +396,9 @@ qlora_status linear_backward(const qlora_nf4& W, const LevelTable& t, const void
         ra.ld3 = mp;
         ra.a3 = o.keep;
         ra.o3_lo = r16;
-        QLORA_TRY(splitk_reduce(ra, s2));
+        QLORA_TRY(rank_product(xl, false, M, K, K, A, K, r, r16, part, sp.u, ra, st, s2));
       }
       // dB = s dY^T U: rows d_out, contraction over tokens, hi and lo columns summed
-      QLORA_TRY(tc_lora_gemm(dY, true, N, M, N, ut, mp, 2 * r16, 2 * r16, part, sp.db, st, s2));
       {
         ReduceArgs ra = reduce_args(part, sp.db, N, r, 2 * r16);
         ra.lo = r16;
@@ -391,10 +406,10 @@ qlora_status linear_backward(const qlora_nf4& W, const LevelTable& t, const void
         ra.ld1 = r;
         ra.a1 = sc;
         ra.acc1 = accumulate;
-        QLORA_TRY(splitk_reduce(ra, s2));
+        QLORA_TRY(rank_product(dY, true, N, M, N, ut, mp, 2 * r16, 2 * r16, part, sp.db, ra, st,
+                               s2));
       }
       // dA = s V^T X: rows d_in, stored transposed as r x d_in
-      QLORA_TRY(tc_lora_gemm(xl, true, K, M, K, vt, mp, 2 * r16, 2 * r16, part, sp.da, st, s2));
       ReduceArgs ra = reduce_args(part, sp.da, K, r, 2 * r16);
       ra.lo = r16;
       ra.o1 = dA;
@@ -402,7 +417,7 @@ qlora_status linear_backward(const qlora_nf4& W, const LevelTable& t, const void
       ra.trans1 = true;
       ra.a1 = sc * o.keep;
       ra.acc1 = accumulate;
-      return splitk_reduce(ra, s2);
+      return rank_product(xl, true, K, M, K, vt, mp, 2 * r16, 2 * r16, part, sp.da, ra, st, s2);
     };
     auto main_work = [&]() -> qlora_status {
       // dX = dY W + sV A in one kernel (split over d_out when needed)

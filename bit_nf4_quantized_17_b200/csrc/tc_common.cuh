@@ -58,5 +58,33 @@ static __device__ __forceinline__ void block_tables(const float (&lv)[16], float
   }
 }
 
+// The outputs of a reduced rank-r product v at row i, column j:
+//   o1  fp32  a1 * v, at [i][j] or transposed [j][i], optionally added to o1
+//   o2  bf16  hi = bf16(a2 v) at [i][j] and, if o2_lo > 0, lo = bf16(a2 v - hi) at [i][j + o2_lo]
+//   o3  bf16  the same pair transposed: hi at [j][i], lo at [j + o3_lo][i]
+// hi + lo carries a2 v to about 16 significant bits through bf16 tensor-core operands.
+static __device__ __forceinline__ void reduce_store(float v, int64_t i, int j, float* o1,
+                                                    int64_t ld1, int trans1, float a1, int acc1,
+                                                    __nv_bfloat16* o2, int64_t ld2, float a2,
+                                                    int o2_lo, __nv_bfloat16* o3, int64_t ld3,
+                                                    float a3, int o3_lo) {
+  if (o1) {
+    float* dst = trans1 ? o1 + j * ld1 + i : o1 + i * ld1 + j;
+    *dst = acc1 ? *dst + a1 * v : a1 * v;
+  }
+  if (o2) {
+    const float x = a2 * v;
+    const __nv_bfloat16 h = __float2bfloat16_rn(x);
+    o2[i * ld2 + j] = h;
+    if (o2_lo) o2[i * ld2 + j + o2_lo] = __float2bfloat16_rn(x - __bfloat162float(h));
+  }
+  if (o3) {
+    const float x = a3 * v;
+    const __nv_bfloat16 h = __float2bfloat16_rn(x);
+    o3[j * ld3 + i] = h;
+    if (o3_lo) o3[(j + o3_lo) * ld3 + i] = __float2bfloat16_rn(x - __bfloat162float(h));
+  }
+}
+
 }  // namespace tc
 }  // namespace qlora
