@@ -53,6 +53,7 @@ struct RankArgs {
   int32_t kt_total;      // 64-wide k-tiles of the whole contraction
   int32_t k_tiles;       // k-tiles per split
   int32_t a_mn;          // A stored MN-major (its rows contiguous)
+  int32_t b_mn;          // B stored MN-major (its n_cols columns contiguous): bn / 64 boxes
   int32_t bn;            // MMA N: columns of the partial tile (multiple of 16, <= 256)
   int32_t b_bytes, stage_bytes, stages, tmem_cols;
   int32_t red_ld;        // fp32 row stride of the shared-memory partial tile
@@ -122,7 +123,13 @@ rank_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       } else {
         ptx::tma_load_2d(&tmA, &full[s], sa, kg * 64, m0);
       }
-      ptx::tma_load_2d(&tmB, &full[s], sa + kABytes, kg * 64, n0);
+      if (p.b_mn) {
+        // B^T tiles: 64 contraction rows x 64 columns, one per 64 columns
+        for (int h = 0; h < p.bn / 64; ++h)
+          ptx::tma_load_2d(&tmB, &full[s], sa + kABytes + h * 8192, n0 + 64 * h, kg * 64);
+      } else {
+        ptx::tma_load_2d(&tmB, &full[s], sa + kABytes, kg * 64, n0);
+      }
       ++issued;
     }
     // never leave with copies in flight into this CTA's shared memory
@@ -130,7 +137,7 @@ rank_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       ptx::mbar_wait(&full[i % p.stages], (i / p.stages) & 1, kTimeoutCycles, nullptr);
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------ MMA issuer
-    const uint32_t idesc = ptx::idesc_bf16(128, p.bn, p.a_mn, 0);
+    const uint32_t idesc = ptx::idesc_bf16(128, p.bn, p.a_mn, p.b_mn);
     for (int i = 0; i < kn; ++i) {
       const int s = i % p.stages;
       const uint32_t ph = (i / p.stages) & 1;
@@ -142,8 +149,9 @@ rank_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       for (int ks = 0; ks < 4; ++ks) {
         const uint64_t ad = p.a_mn ? ptx::sw128_desc(a_addr + ks * 2048, 8192, 1024)
                                    : ptx::sw128_desc(a_addr + ks * 32, 16, 1024);
-        ptx::umma_bf16(tmem, ad, ptx::sw128_desc(b_addr + ks * 32, 16, 1024), idesc,
-                       (i | ks) != 0 ? 1u : 0u);
+        const uint64_t bd = p.b_mn ? ptx::sw128_desc(b_addr + ks * 2048, 8192, 1024)
+                                   : ptx::sw128_desc(b_addr + ks * 32, 16, 1024);
+        ptx::umma_bf16(tmem, ad, bd, idesc, (i | ks) != 0 ? 1u : 0u);
       }
       ptx::umma_commit(&empty[s]);
     }
@@ -282,14 +290,17 @@ int tc_rank_splits(int64_t m_tiles, int64_t k_tiles) {
 }
 
 qlora_status tc_rank_gemm(const void* A, bool a_mn, int64_t m_rows, int64_t kdim, int64_t ld_a,
-                          const void* B, int64_t ld_b, int32_t b_rows, int32_t n_cols,
+                          const void* B, bool b_mn, int64_t ld_b, int32_t b_rows, int32_t n_cols,
                           const ReduceArgs& out, DeviceStatus* st, cudaStream_t s) {
   if (!tc_rank_eligible(n_cols, out.cols, out.lo) || m_rows < 1 || kdim < 1)
     return QLORA_ERR_UNSUPPORTED;
+  // an MN-major B is read in 64-column boxes: n_cols a multiple of 64
+  if (b_mn && n_cols % 64 != 0) return QLORA_ERR_UNSUPPORTED;
   CUtensorMap ma, mb;
   bool ok = a_mn ? make_map(&ma, A, true, m_rows, kdim, ld_a, 64, 64, true)
                  : make_map(&ma, A, true, kdim, m_rows, ld_a, 64, 128, true);
-  ok = ok && make_map(&mb, B, true, kdim, b_rows, ld_b, 64, n_cols, true);
+  ok = ok && (b_mn ? make_map(&mb, B, true, b_rows, kdim, ld_b, 64, 64, true)
+                   : make_map(&mb, B, true, kdim, b_rows, ld_b, 64, n_cols, true));
   if (!ok) return QLORA_ERR_CUDA;
   RankArgs p{};
   p.m_rows = static_cast<int32_t>(m_rows);
@@ -298,6 +309,7 @@ qlora_status tc_rank_gemm(const void* A, bool a_mn, int64_t m_rows, int64_t kdim
   int splits = tc_rank_splits(m_tiles, p.kt_total);
   p.k_tiles = static_cast<int32_t>(ceil_div(p.kt_total, splits));
   p.a_mn = a_mn ? 1 : 0;
+  p.b_mn = b_mn ? 1 : 0;
   p.bn = n_cols;
   p.b_bytes = n_cols * 128;
   p.stage_bytes = kABytes + p.b_bytes;
@@ -311,9 +323,24 @@ qlora_status tc_rank_gemm(const void* A, bool a_mn, int64_t m_rows, int64_t kdim
   const size_t red_bytes = static_cast<size_t>(128) * p.red_ld * sizeof(float);
   const size_t stage_area = static_cast<size_t>(p.stages) * p.stage_bytes;
   const size_t smem = 1024 + (stage_area > red_bytes ? stage_area : red_bytes) + 256;
-  const qlora_status cs =
-      ensure_smem(reinterpret_cast<const void*>(rank_gemm_kernel), static_cast<int>(smem));
+  if (smem > 200 * 1024) return QLORA_ERR_UNSUPPORTED;
+  // the limit is raised once to what any launch of this kernel may use, so
+  // that the occupancy query below prices this launch's own size
+  const qlora_status cs = ensure_smem(reinterpret_cast<const void*>(rank_gemm_kernel), 200 * 1024);
   if (cs != QLORA_OK) return cs;
+  // the largest shared-memory carveout, so that two CTAs fit on an SM (the
+  // driver would otherwise size the carveout for one) - once per device
+  constexpr int kCarveoutTag = 2;
+  int carve = 0;
+  if (!cached_value(reinterpret_cast<const void*>(rank_gemm_kernel), kCarveoutTag, &carve)) {
+    if (cudaFuncSetAttribute(reinterpret_cast<const void*>(rank_gemm_kernel),
+                             cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return QLORA_ERR_CUDA;
+    }
+    store_value(reinterpret_cast<const void*>(rank_gemm_kernel), kCarveoutTag, 1);
+  }
   if (m_tiles > 65535) return QLORA_ERR_SHAPE;
   cudaLaunchConfig_t cfg{};
   cudaLaunchAttribute attr[1];

@@ -102,8 +102,10 @@ struct ReduceArgs;
 // (tc_rank_eligible); otherwise QLORA_ERR_UNSUPPORTED.
 bool tc_rank_eligible(int32_t n_cols, int32_t cols, int32_t lo);
 int tc_rank_splits(int64_t m_tiles, int64_t k_tiles);
+// b_mn: B stored with its n_cols columns contiguous (element (j, k) at
+// k * ld_b + j, b_rows = n_cols); needs n_cols % 64 == 0.
 qlora_status tc_rank_gemm(const void* A, bool a_mn, int64_t m_rows, int64_t kdim, int64_t ld_a,
-                          const void* B, int64_t ld_b, int32_t b_rows, int32_t n_cols,
+                          const void* B, bool b_mn, int64_t ld_b, int32_t b_rows, int32_t n_cols,
                           const ReduceArgs& out, DeviceStatus* st, cudaStream_t s);
 
 struct ReduceArgs {

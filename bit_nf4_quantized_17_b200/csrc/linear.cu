@@ -13,12 +13,13 @@
 //             backward  V = dY B in one launch (V, sV), dX by the CUDA-core GEMV
 //                       (M <= 2, clustered row chunks + one reduce) or by the
 //                       single-CTA fused kernel (split + reduce), then dB and dA
-//   M > 16    forward   U-GEMM (split-K) -> reduce (U fp32, sU bf16) -> fused
-//                       dequant GEMM (CTA pairs for large M) with the LoRA term
-//                       as extra K stages                                 3 launches
-//             backward  B^T, V-GEMM -> reduce (sV, V^T), fused dX GEMM on the
-//                       caller's stream; U^T, dB-GEMM -> reduce, dA-GEMM ->
-//                       reduce on a second stream that joins back        8-9 launches
+//   M > 16    forward   U = X A^T (one cluster-reduced launch: U fp32, sU bf16)
+//                       -> fused dequant GEMM (CTA pairs for large M) with the
+//                       LoRA term as extra K stages                       2 launches
+//             backward  V = dY B (one launch: sV, V^T; B read in place), fused
+//                       dX GEMM on the caller's stream; U^T, dB, dA (one
+//                       launch each) on a second stream that joins back   5 launches
+//             (ranks above 128 keep the split-K GEMM + reduce pairs and B^T)
 // Several adapters per batch and LoRA dropout use the same kernels (LoraOpts).
 // Other shapes take the CUDA-core contraction of gemm_simt.cu.
 #include <algorithm>
@@ -160,7 +161,7 @@ qlora_status rank_product(const void* A, bool a_mn, int64_t m_rows, int64_t kdim
                           float* part, int splits, const ReduceArgs& out, DeviceStatus* st,
                           cudaStream_t s) {
   if (tc_rank_eligible(n_cols, out.cols, out.lo))
-    return tc_rank_gemm(A, a_mn, m_rows, kdim, ld_a, B, ld_b, b_rows, n_cols, out, st, s);
+    return tc_rank_gemm(A, a_mn, m_rows, kdim, ld_a, B, false, ld_b, b_rows, n_cols, out, st, s);
   qlora_status e = tc_lora_gemm(A, a_mn, m_rows, kdim, ld_a, B, ld_b, b_rows, n_cols, part,
                                 splits, st, s);
   if (e != QLORA_OK) return e;
@@ -353,9 +354,12 @@ qlora_status linear_backward(const qlora_nf4& W, const LevelTable& t, const void
     char* sv = ws + L.sv;
     char* vt = ws + L.vt;
     float* part = reinterpret_cast<float*>(ws + L.part_b);
-    // B^T (r x N) so that V = dY B contracts two K-major operands
-    QLORA_TRY(transpose_to_bf16(B, false, N, r, r, bt, N, 0, s));
-    // V = dY B -> sV = s V as [hi | lo] and V^T as [hi ; lo]
+    // V = dY B -> sV = s V as [hi | lo] and V^T as [hi ; lo].  B (N x r, its
+    // r columns contiguous) is read in place as an MN-major operand when r16
+    // is a multiple of 64; otherwise B^T (r x N) is formed first so that both
+    // operands are K-major
+    const bool v_direct = r16 % 64 == 0 && tc_rank_eligible(r16, r, 0);
+    if (!v_direct) QLORA_TRY(transpose_to_bf16(B, false, N, r, r, bt, N, 0, s));
     {
       ReduceArgs ra = reduce_args(part, sp.v, M, r, r16);
       ra.seg = seg;  // U / V: each token keeps only its adapter's columns
@@ -374,7 +378,11 @@ qlora_status linear_backward(const qlora_nf4& W, const LevelTable& t, const void
       ra.ld3 = mp;
       ra.a3 = 1.0f;
       ra.o3_lo = r16;
-      QLORA_TRY(rank_product(dY, false, M, N, N, bt, N, r, r16, part, sp.v, ra, st, s));
+      if (v_direct) {
+        QLORA_TRY(tc_rank_gemm(dY, false, M, N, N, B, true, r, r, r16, ra, st, s));
+      } else {
+        QLORA_TRY(rank_product(dY, false, M, N, N, bt, N, r, r16, part, sp.v, ra, st, s));
+      }
     }
     // dB and dA on the side stream, dX on the caller's: they share only
     // inputs, and the side stream reuses `part` after V's reduction
