@@ -145,14 +145,16 @@ rank_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       ptx::tc_fence_after();
       const uint32_t a_addr = ptx::smem_u32(smem + s * p.stage_bytes);
       const uint32_t b_addr = a_addr + kABytes;
+      // descriptors stepped by their 16-byte address field (see gemm_tc2.cu)
+      const uint64_t a0 = p.a_mn ? ptx::sw128_desc(a_addr, 8192, 1024)
+                                 : ptx::sw128_desc(a_addr, 16, 1024);
+      const uint64_t b0 = p.b_mn ? ptx::sw128_desc(b_addr, 8192, 1024)
+                                 : ptx::sw128_desc(b_addr, 16, 1024);
+      const uint64_t a_step = p.a_mn ? (2048 >> 4) : (32 >> 4);
+      const uint64_t b_step = p.b_mn ? (2048 >> 4) : (32 >> 4);
 #pragma unroll
-      for (int ks = 0; ks < 4; ++ks) {
-        const uint64_t ad = p.a_mn ? ptx::sw128_desc(a_addr + ks * 2048, 8192, 1024)
-                                   : ptx::sw128_desc(a_addr + ks * 32, 16, 1024);
-        const uint64_t bd = p.b_mn ? ptx::sw128_desc(b_addr + ks * 2048, 8192, 1024)
-                                   : ptx::sw128_desc(b_addr + ks * 32, 16, 1024);
-        ptx::umma_bf16(tmem, ad, bd, idesc, (i | ks) != 0 ? 1u : 0u);
-      }
+      for (int ks = 0; ks < 4; ++ks)
+        ptx::umma_bf16(tmem, a0 + a_step * ks, b0 + b_step * ks, idesc, (i | ks) != 0 ? 1u : 0u);
       ptx::umma_commit(&empty[s]);
     }
     ptx::umma_commit(accum);

@@ -266,14 +266,27 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const bool a_mn = !ext && p.a_mn;
       const bool b_mn = ext ? (p.b2_mn != 0) : (BMODE == B_DQ_MN);
       const int steps = (ext && ((kt - k_tiles) % p.k2_half) == p.k2_half - 1) ? p.k2_last_steps : 4;
-      for (int ks = 0; ks < steps; ++ks) {
-        const uint64_t bd = b_mn ? ptx::sw128_desc(b_addr + ks * 2048, 8192, 1024)
-                                 : ptx::sw128_desc(b_addr + ks * 32, 16, 1024);
+      // descriptors stepped by their 16-byte address field from one per
+      // operand and stage (see gemm_tc2.cu: building each afresh made the
+      // issuing thread the limit); main k-tiles unrolled
+      const uint64_t a0 = a_mn ? ptx::sw128_desc(a_addr, 8192, 1024) : ptx::sw128_desc(a_addr, 16, 1024);
+      const uint64_t b0 = b_mn ? ptx::sw128_desc(b_addr, 8192, 1024) : ptx::sw128_desc(b_addr, 16, 1024);
+      const uint64_t a_step = a_mn ? (2048 >> 4) : (32 >> 4);
+      const uint64_t b_step = b_mn ? (2048 >> 4) : (32 >> 4);
+      if (steps == 4) {
 #pragma unroll
-        for (int t = 0; t < MT; ++t) {
-          const uint64_t ad = a_mn ? ptx::sw128_desc(a_addr + ks * 2048, 8192, 1024)
-                                   : ptx::sw128_desc(a_addr + t * kABytes + ks * 32, 16, 1024);
-          ptx::umma_bf16(tmem + t * p.bn, ad, bd, ext ? idesc2 : idesc, (kt | ks) != 0 ? 1u : 0u);
+        for (int ks = 0; ks < 4; ++ks) {
+#pragma unroll
+          for (int t = 0; t < MT; ++t)
+            ptx::umma_bf16(tmem + t * p.bn, a0 + a_step * ks + t * (kABytes >> 4), b0 + b_step * ks,
+                           ext ? idesc2 : idesc, (kt | ks) != 0 ? 1u : 0u);
+        }
+      } else {
+        for (int ks = 0; ks < steps; ++ks) {
+#pragma unroll
+          for (int t = 0; t < MT; ++t)
+            ptx::umma_bf16(tmem + t * p.bn, a0 + a_step * ks + t * (kABytes >> 4), b0 + b_step * ks,
+                           ext ? idesc2 : idesc, (kt | ks) != 0 ? 1u : 0u);
         }
       }
       ptx::umma_commit(&empty[s]);
