@@ -111,7 +111,12 @@ def clock_scaled_peak(peaks, clocks):
 # kernel, from one ncu capture, keyed by the SHA-256 (first 16 hex digits) of
 # the sources that define the kernel at capture time.  When those sources
 # change the figure no longer describes the kernel and the line reports null.
-TRAFFIC = {}
+TRAFFIC = {
+    # per launch, averaged over one layer's 7 linears (4 x 8192^2, 2 x 22016 x 8192,
+    # 8192 x 22016) at 2048 tokens, one capture of each shape
+    ("fused_dgrad", "stack_65b"): {"sha": "06ecc7fa656f4309", "bytes_per_launch": 174507081},
+    ("fused_fwd", "stack_65b"): {"sha": "06ecc7fa656f4309", "bytes_per_launch": 157738605},
+}
 KERNEL_SOURCES = {
     "fused_fwd": ("gemm_tc2.cu", "tc_common.cuh", "tc_ptx.cuh"),
     "fused_dgrad": ("gemm_tc2.cu", "tc_common.cuh", "tc_ptx.cuh"),
