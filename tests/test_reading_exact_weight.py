@@ -1,0 +1,51 @@
+"""Why the linear kernels keep the exact compute weight bf16(RN(level * s_hat)).
+
+"QLoRA技术从入门到精通" 3(2) restores each block of W to BF16 before the
+multiplication; the oracle's compute weight is that value, rounded once.  A
+cheaper expansion for the decode-sized kernels would feed the tensor cores the
+unscaled bf16 levels and apply the block scale once to fp32 partial sums per
+64-weight block.  This CPU check (oracle only, no GPU) shows that such a
+product leaves the stated elementwise bar max |y - ref| / (1 + |ref|) <= 1e-2 at
+the 7B down-projection shape with 16 tokens, although its Frobenius error is
+small, while the exact compute weight stays inside it.  So the GPU paths keep
+the exact weight, and the decode kernels pay its expansion cost.
+"""
+
+import numpy as np
+import torch
+
+import oracle
+from bit_nf4_quantized_17_b200 import workloads as WL
+
+MAX_TOL = 1e-2
+
+
+def _bf16(a):
+    return torch.from_numpy(np.asarray(a, np.float32)).to(torch.bfloat16).float().numpy().astype(np.float64)
+
+
+def _max_rel(got, ref):
+    return float(np.max(np.abs(got - ref) / (1.0 + np.abs(ref))))
+
+
+def test_unscaled_bf16_levels_break_the_elementwise_bar_where_the_exact_weight_does_not():
+    shape = WL.WORKLOADS["mlp_11008"].linears[1]          # down: 4096 x 11008
+    N, K, M = shape.d_out, shape.d_in, 16
+    W = WL.weight(shape, 16).float().numpy()
+    qt = oracle.quantize(W, 64, 256)
+    w_exact = oracle.compute_weight(qt).reshape(N, K).astype(np.float64)
+    x = WL.activations(shape, M, 3).float().numpy().astype(np.float64)
+    y_ref = x @ w_exact.T                                   # the oracle's product (fp64)
+
+    # the exact compute weight, fp32-accurate products, bf16 output: inside the bar
+    assert _max_rel(_bf16(y_ref), y_ref) < 0.5 * MAX_TOL
+
+    # unscaled bf16 levels per weight, block scale applied to each block's sum
+    levels = _bf16(oracle.nf4_levels())
+    idx = np.asarray(qt["idx"]).reshape(N, K // 64, 64)
+    s_hat = np.asarray(oracle.block_scales(qt), np.float64).reshape(N, K // 64)
+    partial = np.einsum("nbk,mbk->mnb", levels[idx], x.reshape(M, K // 64, 64), optimize=True)
+    y_cheap = np.einsum("mnb,nb->mn", partial, s_hat, optimize=True)
+    fro = np.linalg.norm(_bf16(y_cheap) - y_ref) / np.linalg.norm(y_ref)
+    assert fro < 2e-2                                       # the Frobenius bar alone would pass
+    assert _max_rel(_bf16(y_cheap), y_ref) > MAX_TOL        # the elementwise bar does not
