@@ -12,10 +12,10 @@
 // (unmerge), or moves a merged weight from one adapter to another.
 //
 // One CTA per 64 x 128 tile of W: the rank-r product is accumulated in fp32
-// registers over 32-rank chunks of A and B staged in shared memory (each
-// thread 4 rows x 8 columns), then the tile's codes are dequantised, the
-// update added and the result rounded once to bf16.  CUDA cores: the update
-// has only r multiply-adds per weight.
+// registers over chunks of up to 32 ranks of A and B staged in shared memory
+// (each thread 4 rows x 8 columns, paired fp32 multiply-adds), then the tile's
+// codes are dequantised, the update added and the result rounded once to bf16.
+// CUDA cores: the update has only r multiply-adds per weight.
 #include "internal.cuh"
 
 namespace qlora {
@@ -31,7 +31,7 @@ __global__ void __launch_bounds__(256)
 merge_kernel(QView w, LevelTable tab, const __nv_bfloat16* win, const __nv_bfloat16* __restrict__ A,
              const __nv_bfloat16* __restrict__ B, int r, float s, __nv_bfloat16* out) {
   __shared__ __align__(16) float as[kRankChunk][kCols];
-  __shared__ float bs[kRows][kRankChunk + 1];
+  __shared__ __align__(16) float bs[kRankChunk][kRows];  // B transposed: a thread's 4 rows in one read
   __shared__ float lv[16];
   const int64_t N = w.rows, K = w.cols;
   const int64_t n0 = static_cast<int64_t>(blockIdx.y) * kRows;
@@ -41,35 +41,50 @@ merge_kernel(QView w, LevelTable tab, const __nv_bfloat16* win, const __nv_bfloa
 #pragma unroll
     for (int j = 0; j < 16; ++j) lv[j] = tab.level[j];  // constant indices: no local copy
   }
-  float acc[4][8];
+  // acc[i][c] holds columns 2c, 2c + 1 of row i: paired fp32 multiply-adds
+  float2 acc[4][4];
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int c = 0; c < 8; ++c) acc[i][c] = 0.0f;
+    for (int c = 0; c < 4; ++c) acc[i][c] = make_float2(0.0f, 0.0f);
 
   for (int j0 = 0; j0 < r; j0 += kRankChunk) {
+    const int nj = min(kRankChunk, r - j0);
     __syncthreads();
-    for (int e = threadIdx.x; e < kRankChunk * kCols; e += 256) {
-      const int jj = e / kCols, c = e % kCols;
-      const int64_t k = k0 + c;
-      as[jj][c] = (j0 + jj < r && k < K) ? __bfloat162float(A[(j0 + jj) * K + k]) : 0.0f;
+    // A rows j0 .. j0 + nj - 1, columns k0 .. k0 + 127: 8 bf16 (16 bytes) per load
+    for (int e = threadIdx.x; e < nj * (kCols / 8); e += 256) {
+      const int jj = e / (kCols / 8), c8 = 8 * (e % (kCols / 8));
+      const int64_t k = k0 + c8;
+      float4 lo = make_float4(0.0f, 0.0f, 0.0f, 0.0f), hi = lo;
+      if (k < K) {  // K is a multiple of 64: the 8 columns are all in or all out
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(A + (j0 + jj) * K + k));
+        lo = make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u),
+                         __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
+        hi = make_float4(__uint_as_float(v.z << 16), __uint_as_float(v.z & 0xffff0000u),
+                         __uint_as_float(v.w << 16), __uint_as_float(v.w & 0xffff0000u));
+      }
+      *reinterpret_cast<float4*>(&as[jj][c8]) = lo;
+      *reinterpret_cast<float4*>(&as[jj][c8 + 4]) = hi;
     }
-    for (int e = threadIdx.x; e < kRows * kRankChunk; e += 256) {
-      const int i = e / kRankChunk, jj = e % kRankChunk;
+    for (int e = threadIdx.x; e < kRows * nj; e += 256) {
+      const int i = e / nj, jj = e % nj;
       const int64_t n = n0 + i;
-      bs[i][jj] = (j0 + jj < r && n < N) ? __bfloat162float(B[n * r + j0 + jj]) : 0.0f;
+      bs[jj][i] = (n < N) ? __bfloat162float(B[n * r + j0 + jj]) : 0.0f;
     }
     __syncthreads();
 #pragma unroll 4
-    for (int jj = 0; jj < kRankChunk; ++jj) {
+    for (int jj = 0; jj < nj; ++jj) {
       const float4 a0 = *reinterpret_cast<const float4*>(&as[jj][8 * tx]);
       const float4 a1 = *reinterpret_cast<const float4*>(&as[jj][8 * tx + 4]);
-      const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float2 a[4] = {make_float2(a0.x, a0.y), make_float2(a0.z, a0.w),
+                           make_float2(a1.x, a1.y), make_float2(a1.z, a1.w)};
+      const float4 b4 = *reinterpret_cast<const float4*>(&bs[jj][4 * ty]);
+      const float b[4] = {b4.x, b4.y, b4.z, b4.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const float b = bs[4 * ty + i][jj];
+        const float2 bb = make_float2(b[i], b[i]);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) acc[i][c] = fmaf(b, a[c], acc[i][c]);
+        for (int c = 0; c < 4; ++c) acc[i][c] = __ffma2_rn(bb, a[c], acc[i][c]);
       }
     }
   }
@@ -103,8 +118,8 @@ merge_kernel(QView w, LevelTable tab, const __nv_bfloat16* win, const __nv_bfloa
     for (int c = 0; c < 8; c += 2) {
       const float w0 = base[c];
       const float w1 = base[c + 1];
-      const __nv_bfloat162 h = __floats2bfloat162_rn(__fadd_rn(w0, __fmul_rn(s, acc[i][c])),
-                                                     __fadd_rn(w1, __fmul_rn(s, acc[i][c + 1])));
+      const __nv_bfloat162 h = __floats2bfloat162_rn(__fadd_rn(w0, __fmul_rn(s, acc[i][c / 2].x)),
+                                                     __fadd_rn(w1, __fmul_rn(s, acc[i][c / 2].y)));
       o[c / 2] = *reinterpret_cast<const uint32_t*>(&h);
     }
     *reinterpret_cast<uint4*>(out + n * K + k) = make_uint4(o[0], o[1], o[2], o[3]);

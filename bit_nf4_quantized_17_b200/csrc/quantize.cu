@@ -46,10 +46,13 @@ constexpr int kMeanFracBits = 32;
 // huge or not finite, the chunk is redone with IEEE division and a comparison
 // against every threshold.
 //
-// Arithmetic form (mostly FMA-pipe work): step = sat((x' - t_c) * 2^126) is
-// 1.0 or 0.0 outside the near band; 2^23 + count + step has the index in its
-// low mantissa bits, and an integer multiply-add places those bits at the
-// weight's nibble (the constant 2^23 bits cancel: see kPackBias).
+// Arithmetic form (mostly FMA-pipe work, pairs of weights in the paired fp32
+// instructions): the cell's bits, c + 1.5 * 2^23, times the table's row pitch
+// are its shared-memory address less a constant, one integer multiply-add;
+// step = sat((x' - t_c) * 2^126) is 1.0 or 0.0 outside the near band;
+// 2^23 + count + step has the index in its low mantissa bits, and an integer
+// multiply-add places those bits at the weight's nibble (the constant 2^23
+// bits cancel: see kPackBias).
 constexpr int kCells = 65;
 constexpr double kCellPad = 1e-6;
 constexpr float kNear = 1e-6f;
@@ -161,7 +164,9 @@ quantize_blocks_kernel(const T* __restrict__ w, int64_t n, LevelTable tab, CellL
   __syncthreads();
 
   const int lane = threadIdx.x & 31;
-  const float2* my_lut = lut + lane;
+  // address of entry c of this lane's copy: bits(1.5 * 2^23 + c) * 256 + lut_bias
+  // (mod 2^32), since bits(1.5 * 2^23) * 256 = 0x4B400000 * 256 = 0x40000000 mod 2^32
+  const uint32_t lut_bias = static_cast<uint32_t>(__cvta_generic_to_shared(lut + lane)) - 0x40000000u;
   const int64_t n_chunks = (n + E - 1) / E;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   float seen = 0.0f;  // largest finite scale
@@ -193,23 +198,33 @@ quantize_blocks_kernel(const T* __restrict__ w, int64_t n, LevelTable tab, CellL
     uint32_t packed[W];
     bool exact = !(s >= 0x1p-126f && s < 0x1p126f);
     if (!exact) {
-      // |v| <= s and s normal: |x'| <= 1 + 2^-23, so c is within [0, 64];
-      // the clamp below only keeps the shared-memory index in range regardless
+      // |v| <= s (s is the block's absmax, finite) and s normal: |x'| <= 1 + 2^-23,
+      // so f = RN(32 x' + 1.5 * 2^23 + 32) is an integer in [0, 64] above
+      // 1.5 * 2^23 and every table read stays inside this lane's 65 entries
       const float r = __frcp_rn(s);
+      const float2 r2 = make_float2(r, r);
       float near = 1.0f;
 #pragma unroll
       for (int i = 0; i < W; ++i) packed[i] = 0u - kPackBias;
 #pragma unroll
-      for (int j = 0; j < E; ++j) {
-        const float xp = __fmul_rn(v[j], r);
-        const float f = __fmaf_rn(xp, 32.0f, 12582944.0f);  // 1.5 * 2^23 + 32
-        const unsigned int c = min(static_cast<unsigned int>(__float_as_int(f) - 0x4B400000), 64u);
-        const float2 e = my_lut[c * 32];
-        const float d = __fsub_rn(xp, e.x);
-        near = fminf(near, fabsf(d));
-        const float step = __saturatef(__fmul_rn(d, 0x1p126f));
-        const float im = __fadd_rn(e.y, step);  // 2^23 + index
-        packed[j >> 3] += __float_as_uint(im) * (1u << (4 * (j & 7)));
+      for (int j = 0; j < E; j += 2) {
+        const float2 xp = __fmul2_rn(make_float2(v[j], v[j + 1]), r2);
+        const float2 f = __ffma2_rn(xp, make_float2(32.0f, 32.0f),
+                                    make_float2(12582944.0f, 12582944.0f));  // 1.5 * 2^23 + 32
+        float xq[2] = {xp.x, xp.y};
+        const uint32_t fb[2] = {__float_as_uint(f.x), __float_as_uint(f.y)};
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          float tc, below;
+          asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];"
+                       : "=f"(tc), "=f"(below)
+                       : "r"(fb[h] * 256u + lut_bias));
+          const float d = __fsub_rn(xq[h], tc);
+          near = fminf(near, fabsf(d));
+          const float step = __saturatef(__fmul_rn(d, 0x1p126f));
+          const float im = __fadd_rn(below, step);  // 2^23 + index
+          packed[(j + h) >> 3] += __float_as_uint(im) * (1u << (4 * ((j + h) & 7)));
+        }
       }
       exact = near <= kNear;
     }

@@ -115,3 +115,18 @@ def test_unmerge_restores_the_compute_weight():
     upd = s * (np.abs(f64(B)) @ np.abs(f64(A)))
     tol = 2.0 ** -7 * (np.abs(w_bf16) + upd) + 1e-30
     assert np.all(np.abs(f64(back) - w_bf16) <= tol)
+
+
+@pytest.mark.parametrize("N,K,r", [(200, 576, 40), (136, 320, 64), (64, 128, 1)])
+def test_merge_ranks_over_chunks_and_ragged_tiles(N, K, r):
+    # r = 40: one full 32-rank chunk and a partial one; r = 64: two full ones;
+    # N and K leave partial 64-row and 128-column tiles
+    W = WL.randn((N, K), 0.02, 41, torch.bfloat16)
+    A = WL.randn((r, K), 0.3, 42, torch.bfloat16)
+    B = WL.randn((N, r), 0.05, 43, torch.bfloat16)
+    q = Q.qlora_quantize(W.to(DEV))
+    out = Q.qlora_merge(q, A.to(DEV), B.to(DEV), 16.0)
+    torch.cuda.synchronize()
+    w_hat = oracle.dequantize(oracle.quantize(W.float().numpy(), 64, 256)).reshape(N, K)
+    exact = oracle.merge_weight(w_hat, f64(A), f64(B), 16.0)
+    assert _bound_ok(out, exact, np.abs(w_hat.astype(np.float64)), A, B, oracle.lora_scale(16.0, r), r)
