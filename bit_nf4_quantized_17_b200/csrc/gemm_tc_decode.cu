@@ -11,7 +11,9 @@
 // arithmetic itself.  The MMA (tcgen05.mma kind::f16, A from TMEM, M = 128,
 // N = 16) reads the token tile from shared memory (TMA, 128B swizzle).  The
 // LoRA term runs as extension stages with both operands in shared memory
-// (B's rows as A, sU as B).  The contraction is split over CTAs when the
+// (B's rows as A, sU as B): each stage holds a 64-rank B tile once and both
+// the hi and lo halves of sU, and the first two are loaded early, so the
+// term adds no load latency after the main loop.  The contraction is split over CTAs when the
 // rows alone give too few; the splits of a row tile form a thread-block
 // cluster and sum their fp32 tiles in shared memory, in split order, before
 // the one bf16 store of Y.
@@ -42,16 +44,18 @@ constexpr int kXBytes = 2048;                    // 16 token rows x 64 bf16 (128
 constexpr int kCodeBytes = 4096;                 // 128 W rows x 32 bytes
 constexpr int kStageBytes = kXBytes + kCodeBytes;
 constexpr int kExtABytes = 16384;                // 128 rows of B x 64 ranks
-constexpr int kExtBBytes = 2048;                 // 16 tokens x 64 ranks of [hi | lo]
+constexpr int kExtUBytes = 2048;                 // 16 tokens x 64 ranks of sU (its hi or lo half)
+constexpr int kExtSlotBytes = kExtABytes + 2 * kExtUBytes;  // B tile, sU hi, sU lo
+constexpr int kExtSlots = 2;                     // extension stages in flight
 constexpr int kRedBytes = 16 * 128 * 4;          // this CTA's fp32 output tile (cluster reduce)
-constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kExtABytes + kExtBBytes + kRedBytes + 256;
+constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kExtSlots * kExtSlotBytes + kRedBytes + 256;
 constexpr uint32_t kTmemCols = 256;              // D: [0, 16); A slot a: [32 + 32 a, 64 + 32 a)
 constexpr long long kTimeoutCycles = 4000000000ll;
 
 struct DecArgs {
   int32_t m, n;
   int32_t k_tiles, kt_total;  // main k-tiles per split, in all
-  int32_t k2_tiles, k2_half, k2_last_steps;
+  int32_t k2_half, k2_last_steps;  // 64-rank extension stages, MMA steps of the last
   QView w;
   int32_t kblocks;
   int64_t nblocks;
@@ -94,17 +98,16 @@ tc_decode_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  // [kStages x (X | codes)] [ext A | ext B] [output tile] [barriers]
-  uint8_t* ext_a = smem + kStages * kStageBytes;
-  uint8_t* ext_b = ext_a + kExtABytes;
-  float* red = reinterpret_cast<float*>(ext_b + kExtBBytes);  // [16 tokens][128 rows]
-  uint64_t* full = reinterpret_cast<uint64_t*>(ext_b + kExtBBytes + kRedBytes);
+  // [kStages x (X | codes)] [kExtSlots x (B tile | sU hi | sU lo)] [output tile] [barriers]
+  uint8_t* ext = smem + kStages * kStageBytes;
+  float* red = reinterpret_cast<float*>(ext + kExtSlots * kExtSlotBytes);  // [16 tokens][128 rows]
+  uint64_t* full = reinterpret_cast<uint64_t*>(ext + kExtSlots * kExtSlotBytes + kRedBytes);
   uint64_t* empty = full + kStages;   // the stage's MMAs are done
   uint64_t* afull = empty + kStages;  // the slot holds the k-tile's W rows
   uint64_t* aempty = afull + kSlots;  // the slot's MMAs are done
-  uint64_t* ext_full = aempty + kSlots;
-  uint64_t* ext_empty = ext_full + 1;
-  uint64_t* accum = ext_empty + 1;
+  uint64_t* ext_full = aempty + kSlots;       // [kExtSlots]
+  uint64_t* ext_empty = ext_full + kExtSlots;  // [kExtSlots]
+  uint64_t* accum = ext_empty + kExtSlots;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -112,7 +115,7 @@ tc_decode_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
   const int n0 = blockIdx.x * 128;
   const int kt0 = blockIdx.y * p.k_tiles;
   const int kn = min(p.k_tiles, p.kt_total - kt0);
-  const int k2 = (blockIdx.y == 0) ? p.k2_tiles : 0;
+  const int k2 = (blockIdx.y == 0) ? p.k2_half : 0;  // extension stages: 64 ranks each
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -123,8 +126,10 @@ tc_decode_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
       ptx::mbar_init(&afull[a], 4);  // the four warps of the group
       ptx::mbar_init(&aempty[a], 1);
     }
-    ptx::mbar_init(ext_full, 1);
-    ptx::mbar_init(ext_empty, 1);
+    for (int e = 0; e < kExtSlots; ++e) {
+      ptx::mbar_init(&ext_full[e], 1);
+      ptx::mbar_init(&ext_empty[e], 1);
+    }
     ptx::mbar_init(accum, 1);
     *abort_flag = 0;
     ptx::fence_mbar_init();
@@ -146,8 +151,29 @@ tc_decode_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------ TMA producer
-    int issued = 0;
+    // extension stage h: B columns [64 h, 64 h + 64) of this CTA's rows and the
+    // same 64 ranks of sU's hi and lo halves.  sU comes from the launch before
+    // this one, which lets this grid start early (programmatic dependent
+    // launch): the main loop reads only X and W, and the producer waits for
+    // that launch to finish only halfway through it, before the first
+    // extension loads, so they have landed when the main loop ends.
+    auto issue_ext = [&](int h) {
+      const int e = h % kExtSlots;
+      uint8_t* xb = ext + e * kExtSlotBytes;
+      ptx::mbar_arrive_expect_tx(&ext_full[e], kExtSlotBytes);
+      ptx::tma_load_2d(&tmB2, &ext_full[e], xb, h * 64, n0);
+      ptx::tma_load_2d(&tmU2, &ext_full[e], xb + kExtABytes, h * 64, 0);
+      ptx::tma_load_2d(&tmU2, &ext_full[e], xb + kExtABytes + kExtUBytes, (p.k2_half + h) * 64, 0);
+    };
+    int issued = 0, ext_issued = 0;
+    const int early = min(k2, kExtSlots);
+    auto issue_early = [&]() {
+      if (early == 0) return;
+      asm volatile("griddepcontrol.wait;" ::: "memory");  // sU written and visible
+      for (; ext_issued < early; ++ext_issued) issue_ext(ext_issued);
+    };
     bool ok = true;
+    if (kn == 0) issue_early();
     for (int i = 0; i < kn; ++i) {
       const int s = i % kStages;
       const uint32_t ph = (i / kStages) & 1;
@@ -161,20 +187,20 @@ tc_decode_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
       ptx::tma_load_2d(&tmX, &full[s], xs, kg * 64, 0);
       ptx::tma_load_2d(&tmC, &full[s], xs + kXBytes, kg * 32, n0);
       ++issued;
+      if (i == kn / 2) issue_early();
     }
-    int ext_issued = 0;
-    for (int tt = 0; tt < k2 && ok; ++tt) {
-      if (!ptx::mbar_wait(ext_empty, (tt & 1) ^ 1, kTimeoutCycles, abort_flag)) break;
-      const int k2a = tt * 64, k2b = (tt % p.k2_half) * 64;
-      ptx::mbar_arrive_expect_tx(ext_full, kExtABytes + kExtBBytes);
-      ptx::tma_load_2d(&tmB2, ext_full, ext_a, k2b, n0);
-      ptx::tma_load_2d(&tmU2, ext_full, ext_b, k2a, 0);
+    if (ext_issued < early && ok) issue_early();
+    for (int h = ext_issued; h < k2 && ok; ++h) {
+      const int e = h % kExtSlots;
+      if (!ptx::mbar_wait(&ext_empty[e], ((h / kExtSlots) & 1) ^ 1, kTimeoutCycles, abort_flag)) break;
+      issue_ext(h);
       ++ext_issued;
     }
     // never leave with copies in flight into this CTA's shared memory
     for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
       ptx::mbar_wait(&full[i % kStages], (i / kStages) & 1, kTimeoutCycles, nullptr);
-    if (ext_issued > 0) ptx::mbar_wait(ext_full, (ext_issued - 1) & 1, kTimeoutCycles, nullptr);
+    for (int h = (ext_issued > kExtSlots ? ext_issued - kExtSlots : 0); h < ext_issued; ++h)
+      ptx::mbar_wait(&ext_full[h % kExtSlots], (h / kExtSlots) & 1, kTimeoutCycles, nullptr);
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------ MMA issuer
     const uint32_t idesc = ptx::idesc_bf16(128, 16, 0, 0);
@@ -197,16 +223,20 @@ tc_decode_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
       ptx::umma_commit(&empty[s]);   // the stage may be refilled
       ptx::umma_commit(&aempty[a]);  // the slot may be rewritten
     }
-    for (int tt = 0; tt < k2 && ok; ++tt) {
-      if (!ptx::mbar_wait(ext_full, tt & 1, kTimeoutCycles, abort_flag)) break;
+    for (int h = 0; h < k2 && ok; ++h) {
+      const int e = h % kExtSlots;
+      if (!ptx::mbar_wait(&ext_full[e], (h / kExtSlots) & 1, kTimeoutCycles, abort_flag)) break;
       ptx::tc_fence_after();
-      const uint32_t a_addr = ptx::smem_u32(ext_a), b_addr = ptx::smem_u32(ext_b);
-      const int steps = (tt % p.k2_half == p.k2_half - 1) ? p.k2_last_steps : 4;
-      for (int ks = 0; ks < steps; ++ks)
-        ptx::umma_bf16(tmem, ptx::sw128_desc(a_addr + ks * 32, 16, 1024),
-                       ptx::sw128_desc(b_addr + ks * 32, 16, 1024), idesc,
-                       (kn > 0 || tt > 0 || ks > 0) ? 1u : 0u);
-      ptx::umma_commit(ext_empty);
+      const uint32_t a_addr = ptx::smem_u32(ext + e * kExtSlotBytes);
+      const int steps = (h == p.k2_half - 1) ? p.k2_last_steps : 4;
+      for (int part = 0; part < 2; ++part) {  // sU hi, then sU lo, against the same B tile
+        const uint32_t b_addr = a_addr + kExtABytes + part * kExtUBytes;
+        for (int ks = 0; ks < steps; ++ks)
+          ptx::umma_bf16(tmem, ptx::sw128_desc(a_addr + ks * 32, 16, 1024),
+                         ptx::sw128_desc(b_addr + ks * 32, 16, 1024), idesc,
+                         (kn > 0 || h > 0 || part > 0 || ks > 0) ? 1u : 0u);
+      }
+      ptx::umma_commit(&ext_empty[e]);
     }
     ptx::umma_commit(accum);
     ptx::mbar_wait(accum, 0, kTimeoutCycles, nullptr);  // MMAs done before TMEM is freed
@@ -377,7 +407,6 @@ qlora_status tc_decode_forward(const QView& w, const LevelTable& t, const void* 
   p.kt_total = static_cast<int32_t>(K / 64);
   p.k_tiles = static_cast<int32_t>(ceil_div(p.kt_total, splits));
   p.k2_half = (r + 63) / 64;
-  p.k2_tiles = 2 * p.k2_half;
   p.k2_last_steps = ((r - 64 * (p.k2_half - 1)) + 15) / 16;
   p.w = w;
   p.kblocks = static_cast<int32_t>(K / 64);
@@ -394,13 +423,15 @@ qlora_status tc_decode_forward(const QView& w, const LevelTable& t, const void* 
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = static_cast<unsigned>(splits);
-  attr[0].val.clusterDim.z = 1;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // may overlap the U launch
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 1;
+  attr[1].val.clusterDim.y = static_cast<unsigned>(splits);
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = splits > 1 ? 1 : 0;
+  cfg.numAttrs = splits > 1 ? 2 : 1;
   count_launch();
   timing_mark(QLORA_KERNEL_FUSED_FWD, s, true);
   const cudaError_t e = cudaLaunchKernelEx(&cfg, tc_decode_fwd_kernel, mx, mc, mb2, mu2, p, t);

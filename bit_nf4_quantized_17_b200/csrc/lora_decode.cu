@@ -119,6 +119,9 @@ template <int MM>
 __global__ void __launch_bounds__(kThreads)
 rank_down_kernel(const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict__ A, int M,
                  int64_t K, int len, RankOut o) {
+  // the decode forward that follows may start now: it reads this launch's
+  // output only after its own grid-dependency wait
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   __shared__ __align__(16) float xs[MM][kSub];
   __shared__ float red[8][MM];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
