@@ -364,9 +364,10 @@ class Stack:
 
 def time_stack(st, steps, warmup, world, local, peaks, kinds_pass2=True):
     """Warm-up, then `steps` timed steps between CUDA events on the compute
-    stream (barrier + synchronise on both sides); the fused kernels are timed
-    by the library's events inside the timed region, the rank-r GEMMs in a
-    second pass over the same steps.  Returns the measurement dict."""
+    stream (barrier + synchronise on both sides), with no events between the
+    library's launches; then the same steps again with the library's launch
+    events on, for the fused kernels' times, and once more for the rank-r
+    GEMMs'.  Returns the measurement dict."""
     dp, Q, _ = _lib()
     dev = torch.device("cuda", local)
     for i in range(warmup):
@@ -381,17 +382,22 @@ def time_stack(st, steps, warmup, world, local, peaks, kinds_pass2=True):
         barrier(world)
         torch.cuda.synchronize()
         launches0 = Q.qlora_launch_count()
-        Q.qlora_timing_begin((Q.QLORA_KERNEL_FUSED_FWD, Q.QLORA_KERNEL_FUSED_DGRAD),
-                             max_launches=min(65536, 2 * n_lin * steps + 16))
         start.record()
         for i in range(steps):
             st.step(0, world, ev=evs[i])
         end.record()
         launches = Q.qlora_launch_count() - launches0
         torch.cuda.synchronize()
-        kt = Q.qlora_timing_end()
         barrier(world)
     clocks = clk.summary()
+    # per-kernel times in separate passes: a launch event between the rank-r
+    # kernel and the fused kernel would also stop their programmatic overlap
+    Q.qlora_timing_begin((Q.QLORA_KERNEL_FUSED_FWD, Q.QLORA_KERNEL_FUSED_DGRAD),
+                         max_launches=min(65536, 2 * n_lin * steps + 16))
+    for i in range(steps):
+        st.step(0, world)
+    torch.cuda.synchronize()
+    kt = Q.qlora_timing_end()
     if kinds_pass2:
         Q.qlora_timing_begin((Q.QLORA_KERNEL_LORA_GEMM,),
                              max_launches=min(65536, 4 * n_lin * steps + 16))
@@ -573,19 +579,22 @@ def time_single(name, steps, warmup, peaks, dev):
     for i in range(warmup):
         step(sets[i % n_sets])
     torch.cuda.synchronize()
-    kinds = (Q.QLORA_KERNEL_FUSED_FWD, Q.QLORA_KERNEL_FUSED_DGRAD)
-    Q.qlora_timing_begin(kinds, max_launches=4 * len(shapes) * steps + 16)
-    graph = torch.cuda.CUDAGraph()
-    cap = torch.cuda.Stream()
-    cap.wait_stream(torch.cuda.current_stream())
+    def capture():
+        graph = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream()
+        cap.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(cap):
+            with torch.cuda.graph(graph, stream=cap):
+                for i in range(steps):
+                    step(sets[i % n_sets])
+        torch.cuda.current_stream().wait_stream(cap)
+        torch.cuda.synchronize()
+        return graph
+
+    # the timed graph holds the library's launches only (no launch events)
     l0 = Q.qlora_launch_count()
-    with torch.cuda.stream(cap):
-        with torch.cuda.graph(graph, stream=cap):
-            for i in range(steps):
-                step(sets[i % n_sets])
+    graph = capture()
     launches = Q.qlora_launch_count() - l0
-    torch.cuda.current_stream().wait_stream(cap)
-    torch.cuda.synchronize()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(dev.index or 0) as clk:
         torch.cuda.synchronize()
@@ -593,6 +602,14 @@ def time_single(name, steps, warmup, peaks, dev):
         graph.replay()
         end.record()
         torch.cuda.synchronize()
+    del graph
+    # the fused kernels' times from a second graph of the same steps, with the
+    # library's launch events captured into it
+    kinds = (Q.QLORA_KERNEL_FUSED_FWD, Q.QLORA_KERNEL_FUSED_DGRAD)
+    Q.qlora_timing_begin(kinds, max_launches=4 * len(shapes) * steps + 16)
+    graph = capture()
+    graph.replay()
+    torch.cuda.synchronize()
     del graph  # it refers to the library's timing events
     kt = Q.qlora_timing_end()
     Q.qlora_timing_begin((Q.QLORA_KERNEL_QUANTIZE, Q.QLORA_KERNEL_LORA_GEMM),
@@ -727,10 +744,16 @@ def time_decode(peaks, dev, steps=50, warmup=5):
             ms, n = kt[kind]
             if n:
                 avg = ms * 1e-3 / n
+                alu_peak = alu_peak_ops(peaks)
                 fused[name] = {"avg_us": round(avg * 1e6, 2),
                                "gbs": round((wb + extra) / avg / 1e9, 1),
                                "frac_hbm": round((wb + extra) / avg / 1e9 / peaks["hbm"], 4),
-                               "nf4_frac_hbm": round(wb / avg / 1e9 / peaks["hbm"], 4)}
+                               "nf4_frac_hbm": round(wb / avg / 1e9 / peaks["hbm"], 4),
+                               "alu": {"bound": "alu",
+                                       "achieved": round(EXPAND_OPS_PER_WEIGHT * N * K / avg / 1e12, 2),
+                                       "peak": round(alu_peak / 1e12, 2), "unit": "T lane-ops/s",
+                                       "frac": round(EXPAND_OPS_PER_WEIGHT * N * K / avg / alu_peak, 4),
+                                       "ops_per_weight": EXPAND_OPS_PER_WEIGHT}}
         out[f"M{M}"] = {
             "fwd_us": round(t_f * 1e6, 2), "bwd_us": round(t_b * 1e6, 2),
             "fwd_nf4_gbs": round(wb / t_f / 1e9, 1), "bwd_nf4_gbs": round(wb / t_b / 1e9, 1),
@@ -744,6 +767,19 @@ def time_decode(peaks, dev, steps=50, warmup=5):
     out["workload"] = "mlp gate/up 11008x4096, r=64, alpha=16; NF4 bytes per pass " \
                       f"{nf4_bytes(N, K)}; 8 rotating weight copies; median of {steps}"
     return out
+
+
+# Minimum ALU work of the exact compute weight per weight: 21 byte-permute,
+# shift and logic operations per 8 weights for the lookup, and 16 per 64 weights
+# for the block's tables (the conversions and the table permutes)
+EXPAND_OPS_PER_WEIGHT = 21 / 8 + 16 / 64
+
+
+def alu_peak_ops(peaks):
+    """ALU lane-operations per second: 64 lanes per clock on each of the
+    device's SMs at the maximum SM clock."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count if torch.cuda.is_available() else 148
+    return sms * 64 * peaks.get("sm_max_mhz", 1965.0) * 1e6
 
 
 def time_merge(peaks, dev, steps=20):

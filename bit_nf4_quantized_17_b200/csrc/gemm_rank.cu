@@ -64,6 +64,9 @@ struct RankArgs {
 __global__ void __launch_bounds__(kThreads, 1)
 rank_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const RankArgs p) {
+  // the fused GEMM that follows may start now: it reads this launch's output
+  // only after its own grid-dependency wait
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));

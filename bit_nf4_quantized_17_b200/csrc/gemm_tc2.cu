@@ -182,6 +182,10 @@ tc2_fused_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         // extension stage tt: A2 columns [64 tt, 64 tt + 64) of [hi | lo];
         // this CTA's half of B2 at LoRA ranks [64 (tt mod half), ...)
         const int tt = kt - p.kt_total;
+        // A2 (sU or sV) is the output of the launch before this one, which
+        // lets this grid start early (programmatic dependent launch): the
+        // main loop reads only the activations and W
+        if (tt == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
         const int k2a = tt * 64;
         const int k2b = (tt % p.k2_half) * 64;
         if (rank == 0) ptx::mbar_arrive_expect_tx(&full_a[s], 2 * (p.a_bytes + b_bytes));
@@ -377,13 +381,15 @@ qlora_status launch_tc2(const CUtensorMap& ma, const CUtensorMap& mb, const CUte
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // may overlap the U / V launch
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   const int kind = BMODE == B_DQ_K ? QLORA_KERNEL_FUSED_FWD : QLORA_KERNEL_FUSED_DGRAD;
   count_launch();
   timing_mark(kind, s, true);

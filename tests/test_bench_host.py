@@ -6,6 +6,7 @@ import os
 import sys
 
 import pytest
+import torch
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 sys.path.insert(0, ROOT)
@@ -117,3 +118,11 @@ def test_stack_config_names_the_workload():
     c = bench.stack_config("stack_65b", 80, 2)
     assert c["global_batch"] == 8 and c["parallelism"] == "dp2" and c["layers"] == 80
     assert "stack_65b" in c["workload"] and "80 layers" in c["workload"]
+
+
+def test_decode_alu_roofline_constants():
+    # 21 lookup operations per 8 weights plus 16 table operations per 64-weight block,
+    # against 64 ALU lanes per clock per SM at the maximum clock (148 SMs without a GPU)
+    assert bench.EXPAND_OPS_PER_WEIGHT == 21 / 8 + 16 / 64
+    if not torch.cuda.is_available():
+        assert bench.alu_peak_ops({"sm_max_mhz": 1965.0}) == 148 * 64 * 1965.0e6
