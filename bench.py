@@ -114,8 +114,8 @@ def clock_scaled_peak(peaks, clocks):
 TRAFFIC = {
     # per launch, averaged over one layer's 7 linears (4 x 8192^2, 2 x 22016 x 8192,
     # 8192 x 22016) at 2048 tokens, one capture of each shape
-    ("fused_dgrad", "stack_65b"): {"sha": "06ecc7fa656f4309", "bytes_per_launch": 174507081},
-    ("fused_fwd", "stack_65b"): {"sha": "06ecc7fa656f4309", "bytes_per_launch": 157738605},
+    ("fused_dgrad", "stack_65b"): {"sha": "9be4da7b80466d50", "bytes_per_launch": 171768722},
+    ("fused_fwd", "stack_65b"): {"sha": "9be4da7b80466d50", "bytes_per_launch": 157108553},
 }
 KERNEL_SOURCES = {
     "fused_fwd": ("gemm_tc2.cu", "tc_common.cuh", "tc_ptx.cuh"),
