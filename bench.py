@@ -1077,6 +1077,15 @@ def run_case(args):
     dB = torch.empty((N, r), dtype=torch.float32, device=dev)
     torch.cuda.synchronize()
     t = 0.0
+    if args.merge:  # the adapter merged into a restored bf16 weight instead
+        for _ in range(args.iters):
+            t0 = time.perf_counter()
+            Q.qlora_merge(q, inp["A"], inp["B"], shape.alpha)
+            torch.cuda.synchronize()
+            t = time.perf_counter() - t0
+        print(f"{args.case}[{args.linear}] {N}x{K} r={r}: merge, last iteration {t * 1e6:.1f} us "
+              f"(wall clock, not a benchmark)")
+        return
     for _ in range(args.iters):
         t0 = time.perf_counter()
         Q.qlora_linear_fwd(q, inp["A"], inp["B"], shape.alpha, inp["X"], Y=Y, U_save=U,
@@ -1111,6 +1120,7 @@ def main(argv=None):
     ap.add_argument("--tokens", type=int, default=None)
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--fwd-only", action="store_true")
+    ap.add_argument("--merge", action="store_true", help="with --case: run qlora_merge instead")
     ap.add_argument("--cpu-configs", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.case is None:

@@ -115,7 +115,9 @@ tc_decode_fwd_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_const
   const int n0 = blockIdx.x * 128;
   const int kt0 = blockIdx.y * p.k_tiles;
   const int kn = min(p.k_tiles, p.kt_total - kt0);
-  const int k2 = (blockIdx.y == 0) ? p.k2_half : 0;  // extension stages: 64 ranks each
+  // extension stages (64 ranks each) on the last split, which has the fewest
+  // main k-tiles when they do not divide evenly
+  const int k2 = (blockIdx.y == gridDim.y - 1) ? p.k2_half : 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
