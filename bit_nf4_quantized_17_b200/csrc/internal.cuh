@@ -97,6 +97,15 @@ qlora_status launch_merge(const qlora_nf4& q, const LevelTable& t, const void* A
 // merge.cu: W_out = bf16(W_in + (alpha / r) B A) for a dense bf16 W_in (may alias W_out)
 qlora_status launch_merge_dense(const void* W_in, int64_t rows, int64_t cols, const void* A,
                                 const void* B, int32_t r, float alpha, void* out, cudaStream_t s);
+// The same two updates with the rank-r product on the tensor cores
+// (merge_tc.cu), for r a multiple of 8 up to 256 and cols a multiple of 64.
+struct QView;
+bool merge_tc_eligible(int64_t cols, int32_t r);
+qlora_status launch_merge_tc(const QView& w, const LevelTable& t, const void* A, const void* B,
+                             int32_t r, float alpha, void* out, cudaStream_t s);
+qlora_status launch_merge_dense_tc(const void* W_in, int64_t rows, int64_t cols, const void* A,
+                                   const void* B, int32_t r, float alpha, void* out,
+                                   cudaStream_t s);
 
 // Everything a linear-layer kernel needs to read a quantised W.
 struct QView {

@@ -11,7 +11,10 @@
 // bf16(W_in + s B A): with -alpha it takes a merged adapter out again
 // (unmerge), or moves a merged weight from one adapter to another.
 //
-// One CTA per 64 x 128 tile of W: the rank-r product is accumulated in fp32
+// This file holds the CUDA-core form, for the shapes the tensor-core kernel
+// (merge_tc.cu) does not take: r not a multiple of 8, or cols not a multiple
+// of 64 (dense form).  One CTA per 64 x 128 tile of W: the rank-r product is
+// accumulated in fp32
 // registers over chunks of up to 32 ranks of A and B staged in shared memory
 // (each thread 4 rows x 8 columns, paired fp32 multiply-adds), then the tile's
 // codes are dequantised, the update added and the result rounded once to bf16.
@@ -132,6 +135,7 @@ qlora_status launch_merge(const qlora_nf4& q, const LevelTable& t, const void* A
                           int32_t r, float alpha, void* out, cudaStream_t s) {
   QView w{q.codes, q.scale_codes, q.factors, q.mean, q.rows, q.cols,
           q.dq_blocksize ? __builtin_ctz(q.dq_blocksize) : -1, __builtin_ctz(q.blocksize) - 6};
+  if (merge_tc_eligible(q.cols, r)) return launch_merge_tc(w, t, A, B, r, alpha, out, s);
   const dim3 grid(static_cast<unsigned>(ceil_div(q.cols, kCols)),
                   static_cast<unsigned>(ceil_div(q.rows, kRows)));
   if (grid.y > 65535) return QLORA_ERR_SHAPE;
@@ -147,6 +151,8 @@ qlora_status launch_merge(const qlora_nf4& q, const LevelTable& t, const void* A
 
 qlora_status launch_merge_dense(const void* W_in, int64_t rows, int64_t cols, const void* A,
                                 const void* B, int32_t r, float alpha, void* out, cudaStream_t s) {
+  if (merge_tc_eligible(cols, r))
+    return launch_merge_dense_tc(W_in, rows, cols, A, B, r, alpha, out, s);
   QView w{};
   w.rows = rows;
   w.cols = cols;

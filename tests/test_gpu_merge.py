@@ -130,3 +130,24 @@ def test_merge_ranks_over_chunks_and_ragged_tiles(N, K, r):
     w_hat = oracle.dequantize(oracle.quantize(W.float().numpy(), 64, 256)).reshape(N, K)
     exact = oracle.merge_weight(w_hat, f64(A), f64(B), 16.0)
     assert _bound_ok(out, exact, np.abs(w_hat.astype(np.float64)), A, B, oracle.lora_scale(16.0, r), r)
+
+
+@pytest.mark.parametrize("r", [136, 256])
+def test_merge_ranks_over_several_stages(r):
+    # r = 136: three 64-rank stages, the last with one 16-rank step; r = 256: four
+    # full stages through a two-stage ring; both forms (NF4 base and dense base)
+    N, K = 160, 320
+    W = WL.randn((N, K), 0.02, 51, torch.bfloat16)
+    A = WL.randn((r, K), 0.1, 52, torch.bfloat16)
+    B = WL.randn((N, r), 0.05, 53, torch.bfloat16)
+    Ad, Bd = A.to(DEV), B.to(DEV)
+    q = Q.qlora_quantize(W.to(DEV))
+    out = Q.qlora_merge(q, Ad, Bd, 32.0)
+    dense = Q.qlora_merge_dense(W.to(DEV), Ad, Bd, 32.0)
+    torch.cuda.synchronize()
+    s = oracle.lora_scale(32.0, r)
+    w_hat = oracle.dequantize(oracle.quantize(W.float().numpy(), 64, 256)).reshape(N, K)
+    exact = oracle.merge_weight(w_hat, f64(A), f64(B), 32.0)
+    assert _bound_ok(out, exact, np.abs(w_hat.astype(np.float64)), A, B, s, r)
+    exact_d = oracle.merge_weight(f64(W), f64(A), f64(B), 32.0)
+    assert _bound_ok(dense, exact_d, np.abs(f64(W)), A, B, s, r)
