@@ -246,8 +246,24 @@ rank_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                          static_cast<__nv_bfloat16*>(o.o3), o.ld3, o.a3, o.o3_lo);
       }
     }
-    if (o.o2 && o.o2_pad) {
-      // the padding columns of o2 of this CTA's rows: [cols, o2_lo) and [o2_lo + cols, 2 o2_lo)
+    if (o.o2 && o.o2_pad && (cols % 8) == 0 && (o.o2_lo % 8) == 0 && (o.ld2 % 8) == 0 &&
+        (reinterpret_cast<uintptr_t>(o.o2) & 15) == 0) {
+      // the padding columns of o2 of this CTA's rows, [cols, o2_lo) and
+      // [o2_lo + cols, 2 o2_lo), in 16-byte stores: both runs start and end
+      // on 8-column boundaries
+      const int chunks = (o.o2_lo - cols) / 8;  // per run
+      uint4* o2 = static_cast<uint4*>(o.o2);
+      const int64_t ld16 = o.ld2 / 8;
+      for (int e = tid; e < rows_per * 2 * chunks; e += 128) {
+        const int il = i0 + e / (2 * chunks);
+        const int c = e - (e / (2 * chunks)) * 2 * chunks;
+        const int64_t gi = static_cast<int64_t>(m0) + il;
+        if (gi >= p.m_rows) continue;
+        o2[gi * ld16 + ((c < chunks) ? cols / 8 + c : (o.o2_lo + cols) / 8 + (c - chunks))] =
+            make_uint4(0u, 0u, 0u, 0u);
+      }
+    } else if (o.o2 && o.o2_pad) {
+      // the same, one column at a time
       const int pad = o.o2_lo - cols;
       __nv_bfloat16* o2 = static_cast<__nv_bfloat16*>(o.o2);
       for (int e = tid; e < rows_per * 2 * pad; e += 128) {
