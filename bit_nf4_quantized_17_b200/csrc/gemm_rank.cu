@@ -8,11 +8,11 @@
 // are thin: r <= 256 output columns against a contraction of thousands.  They
 // move X or dY once and are bound by that read.  One launch computes
 // D = A . B^T for 128-row tiles of A: the contraction is split over the S CTAs
-// of a cluster (S = 1, 2, 4 or 8) so that the grid covers the SMs, each CTA
+// of a cluster (S = 1 .. 8) so that the grid covers the SMs, each CTA
 // accumulates its share in TMEM (tcgen05.mma kind::f16, M = 128, N = bn,
 // operands by TMA in 128B-swizzled tiles), and the S fp32 partial tiles are
 // summed in distributed shared memory, in split order (deterministic), by the
-// CTA that owns each slice of rows.  The sums go straight to the outputs the
+// CTA that owns each slice of ceil(128 / S) rows.  The sums go straight to the outputs the
 // callers need (fp32, bf16 [hi | lo] pairs, transposed copies), so no partial
 // reaches global memory and no separate reduce launch follows.
 //
@@ -196,8 +196,10 @@ rank_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   // --------------------------- sum over the splits, in order, and store
   if (warp >= 2) {
     const ReduceArgs& o = p.o;
-    const int rows_per = 128 / static_cast<int>(S);
-    const int i0 = static_cast<int>(z) * rows_per;
+    // this CTA's slice of the 128 rows: ceil(128 / S) rows, the last slice shorter
+    const int slice = (128 + static_cast<int>(S) - 1) / static_cast<int>(S);
+    const int i0 = static_cast<int>(z) * slice;
+    const int rows_per = max(0, min(slice, 128 - i0));
     const int cols = o.cols;
     const int tid = threadIdx.x - 64;
     uint32_t peer[8];
@@ -303,11 +305,14 @@ int tc_rank_splits(int64_t m_tiles, int64_t k_tiles) {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     (void)cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // about two CTAs per SM in one wave; at least 8 k-tiles per split so that
-  // each CTA streams
-  int s = 1;
-  while (s < 8 && m_tiles * (2 * s) <= 2 * sms && k_tiles >= 8 * (2 * s)) s <<= 1;
-  return s;
+  // clustered launches run about one CTA per SM: as many splits as give one
+  // CTA per SM in one wave, at least 8 k-tiles per split, at most 8 (a
+  // cluster holds the splits)
+  int64_t s = m_tiles > 0 ? sms / m_tiles : 1;
+  if (s > 8) s = 8;
+  if (s > k_tiles / 8) s = k_tiles / 8;
+  if (s < 1) s = 1;
+  return static_cast<int>(s);
 }
 
 qlora_status tc_rank_gemm(const void* A, bool a_mn, int64_t m_rows, int64_t kdim, int64_t ld_a,
@@ -383,7 +388,7 @@ qlora_status tc_rank_gemm(const void* A, bool a_mn, int64_t m_rows, int64_t kdim
       break;
     }
     if (static_cast<int64_t>(resident) >= m_tiles) break;
-    splits >>= 1;
+    splits -= 1;
   }
   p.k_tiles = static_cast<int32_t>(ceil_div(p.kt_total, splits));
   cfg.gridDim = dim3(1u, static_cast<unsigned>(m_tiles), static_cast<unsigned>(splits));
