@@ -305,10 +305,11 @@ int tc_rank_splits(int64_t m_tiles, int64_t k_tiles) {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     (void)cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // clustered launches run about one CTA per SM: as many splits as give one
-  // CTA per SM in one wave, at least 8 k-tiles per split, at most 8 (a
-  // cluster holds the splits)
-  int64_t s = m_tiles > 0 ? sms / m_tiles : 1;
+  // up to two CTAs per SM in one wave, at least 8 k-tiles per split, at most
+  // 8 (a cluster holds the splits); the launch steps down from there while
+  // the clusters would not all be resident (large clusters run about one CTA
+  // per SM, small ones two)
+  int64_t s = m_tiles > 0 ? (2 * static_cast<int64_t>(sms)) / m_tiles : 1;
   if (s > 8) s = 8;
   if (s > k_tiles / 8) s = k_tiles / 8;
   if (s < 1) s = 1;

@@ -355,10 +355,11 @@ qlora_status linear_backward(const qlora_nf4& W, const LevelTable& t, const void
     char* vt = ws + L.vt;
     float* part = reinterpret_cast<float*>(ws + L.part_b);
     // V = dY B -> sV = s V as [hi | lo] and V^T as [hi ; lo].  B (N x r, its
-    // r columns contiguous) is read in place as an MN-major operand when r16
-    // is a multiple of 64; otherwise B^T (r x N) is formed first so that both
-    // operands are K-major
-    const bool v_direct = r16 % 64 == 0 && tc_rank_eligible(r16, r, 0);
+    // r columns contiguous) is read in place as an MN-major operand, in boxes
+    // of 64 columns (the MMA is lora_span(r) wide; columns past r read as 0),
+    // when its rows are a multiple of 16 bytes; otherwise B^T (r x N) is
+    // formed first so that both operands are K-major
+    const bool v_direct = r % 8 == 0 && tc_rank_eligible(span, r, 0);
     if (!v_direct) QLORA_TRY(transpose_to_bf16(B, false, N, r, r, bt, N, 0, s));
     {
       ReduceArgs ra = reduce_args(part, sp.v, M, r, r16);
@@ -379,7 +380,7 @@ qlora_status linear_backward(const qlora_nf4& W, const LevelTable& t, const void
       ra.a3 = 1.0f;
       ra.o3_lo = r16;
       if (v_direct) {
-        QLORA_TRY(tc_rank_gemm(dY, false, M, N, N, B, true, r, r, r16, ra, st, s));
+        QLORA_TRY(tc_rank_gemm(dY, false, M, N, N, B, true, r, r, span, ra, st, s));
       } else {
         QLORA_TRY(rank_product(dY, false, M, N, N, bt, N, r, r16, part, sp.v, ra, st, s));
       }
