@@ -232,6 +232,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         const int tt = kt - k_tiles;
         const int k2a = tt * 64;
         const int k2b = (tt % p.k2_half) * 64;
+        // A2 (sU or sV) is the output of the launch before this one, which
+        // lets the fused kernels start early (programmatic dependent launch):
+        // the main loop reads only the activations and W
+        if (tt == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
         ptx::mbar_arrive_expect_tx(&full_a[s], p.a_bytes + 32768);
         ptx::tma_load_2d(&tmA2, &full_a[s], sa, k2a, m0);
         if (p.b2_mn) {
@@ -590,7 +594,27 @@ qlora_status launch_tc(const CUtensorMap& a, const CUtensorMap& b, const CUtenso
                        : BMODE == B_DQ_K ? QLORA_KERNEL_FUSED_FWD
                                          : QLORA_KERNEL_FUSED_DGRAD;
   timing_mark(kind, s, true);
-  tc_gemm_kernel<BMODE, STAGES, MT><<<grid, kThreads, smem, s>>>(a, b, a2, b2, p, t);
+  if constexpr (BMODE == B_TMA_K) {
+    tc_gemm_kernel<BMODE, STAGES, MT><<<grid, kThreads, smem, s>>>(a, b, a2, b2, p, t);
+  } else {
+    // the fused kernels read the previous launch's output only in their LoRA
+    // stages: they may start while it runs
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, tc_gemm_kernel<BMODE, STAGES, MT>, a, b, a2, b2, p, t) !=
+        cudaSuccess) {
+      timing_mark(kind, s, false);
+      return QLORA_ERR_CUDA;
+    }
+  }
   timing_mark(kind, s, false);
   return after_launch(BMODE == B_TMA_K ? "tc_gemm(lora)" : BMODE == B_DQ_K ? "tc_gemm(fwd)" : "tc_gemm(dgrad)", s);
 }

@@ -117,6 +117,10 @@ gemv_dgrad_kernel(QView w, LevelTable tab, const __nv_bfloat16* __restrict__ dY,
 #pragma unroll
     for (int e = 0; e < 32; ++e) red[(warp * MM + m) * kRedStride + lane * 33 + e] = acc[m][e];
   __syncthreads();
+  // V is the output of the launch before this one, which lets this grid
+  // start early (programmatic dependent launch): the row loop above reads only
+  // dY and W
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   constexpr int kPer = MM * 1024 / kThreads;  // column sums per thread
   float tv[kPer];
 #pragma unroll
@@ -196,13 +200,15 @@ qlora_status gemv_dgrad(const QView& w, const LevelTable& t, const void* dY, int
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = kCluster;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // may overlap the V launch
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   // as many row chunks as keep every cluster resident at once (one wave),
   // within the workspace's bound
   const void* fn = reinterpret_cast<const void*>(kernel);

@@ -178,6 +178,9 @@ template <int MM>
 __global__ void __launch_bounds__(kThreads)
 rank_v_kernel(const __nv_bfloat16* __restrict__ dY, const __nv_bfloat16* __restrict__ B, int M,
               int64_t N, int len, RankOut o) {
+  // the dX kernel that follows may start now: it reads V only after its own
+  // grid-dependency wait
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   constexpr int JB = MM >= 8 ? 4 : 8;
   constexpr int kAhead = MM >= 8 ? 2 : 4;
   __shared__ float wred[8][MM * JB];
