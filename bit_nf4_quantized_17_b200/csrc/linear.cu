@@ -19,7 +19,11 @@
 //             backward  V = dY B (one launch: sV, V^T; B read in place), fused
 //                       dX GEMM on the caller's stream; U^T, dB, dA (one
 //                       launch each) on a second stream that joins back   5 launches
-//             (ranks above 128 keep the split-K GEMM + reduce pairs and B^T)
+//             (ranks above 128 keep the split-K GEMM + reduce pairs for dB, dA)
+// Every kernel that reads U or V right after the launch that makes it (the
+// fused GEMMs, the decode kernel, the dX GEMV) is launched as its programmatic
+// dependent: it reads them only after a grid-dependency wait, late in the
+// kernel, so it starts while the U / V launch still runs.
 // Several adapters per batch and LoRA dropout use the same kernels (LoraOpts).
 // Other shapes take the CUDA-core contraction of gemm_simt.cu.
 #include <algorithm>
@@ -356,9 +360,10 @@ qlora_status linear_backward(const qlora_nf4& W, const LevelTable& t, const void
     float* part = reinterpret_cast<float*>(ws + L.part_b);
     // V = dY B -> sV = s V as [hi | lo] and V^T as [hi ; lo].  B (N x r, its
     // r columns contiguous) is read in place as an MN-major operand, in boxes
-    // of 64 columns (the MMA is lora_span(r) wide; columns past r read as 0),
-    // when its rows are a multiple of 16 bytes; otherwise B^T (r x N) is
-    // formed first so that both operands are K-major
+    // of 64 columns (the MMA is lora_span(r) wide; columns past r read as 0);
+    // its rows are a multiple of 16 bytes on this path (r % 8 == 0).  The B^T
+    // form below (both operands K-major) is kept for any shape the rank
+    // kernel would refuse
     const bool v_direct = r % 8 == 0 && tc_rank_eligible(span, r, 0);
     if (!v_direct) QLORA_TRY(transpose_to_bf16(B, false, N, r, r, bt, N, 0, s));
     {
