@@ -221,7 +221,10 @@ qlora_status qlora_linear_bwd_multi(const qlora_nf4* W, const void* A, const voi
  * written; 16-byte aligned).  Requirements as for qlora_linear_fwd (W->cols a
  * multiple of W->blocksize, 1 <= r <= 256); errors QLORA_ERR_NULL, _ALIGN,
  * _SHAPE, _UNSUPPORTED, _CUDA.  Stream-ordered; allocates nothing.  The
- * result can be quantised again with qlora_quantize. */
+ * result can be quantised again with qlora_quantize.  For r a multiple of 8 the
+ * rank-r product runs on the tensor cores; its device-side waits are bounded,
+ * and as the call takes no status word, a wait that gives up (it does not in
+ * correct operation) leaves NaN in its 128 x 256 tile of W_out. */
 qlora_status qlora_merge(const qlora_nf4* W, const void* A, const void* B, int32_t r,
                          float alpha, void* W_out, void* stream);
 
@@ -231,7 +234,9 @@ qlora_status qlora_merge(const qlora_nf4* W, const void* A, const void* B, int32
  * one adapter to another.  Device buffers: W_in and W_out (rows x cols bf16,
  * row-major; W_out may be W_in: in place), A (r x cols bf16), B (rows x r
  * bf16), all 16-byte aligned.  Errors: QLORA_ERR_NULL, _ALIGN, _SHAPE (rows or
- * cols < 1, cols % 8 != 0, r outside [1, 256], rows > 2^22), _CUDA. */
+ * cols < 1, cols % 8 != 0, r outside [1, 256], rows > 2^22), _CUDA.  With r a
+ * multiple of 8 and cols a multiple of 64 it takes the tensor-core form, with
+ * the same NaN-tile behaviour as qlora_merge on a wait that gives up. */
 qlora_status qlora_merge_dense(const void* W_in, int64_t rows, int64_t cols, const void* A,
                                const void* B, int32_t r, float alpha, void* W_out, void* stream);
 
