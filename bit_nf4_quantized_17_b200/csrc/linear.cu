@@ -10,9 +10,10 @@
 //   M <= 16   forward   U = X A^T in one cluster-reduced launch (U_save, sU),
 //                       then the decode kernel with W in TMEM; its contraction
 //                       splits are summed in their cluster             2 launches
-//             backward  V = dY B in one launch (V, sV), dX by the CUDA-core GEMV
+//             backward  V = dY B in one launch (V, sV); dX by the CUDA-core GEMV
 //                       (M <= 2, clustered row chunks + one reduce) or by the
-//                       single-CTA fused kernel (split + reduce), then dB and dA
+//                       single-CTA fused kernel (split + reduce); dB, dA on a
+//                       second stream that joins back
 //   M > 16    forward   U = X A^T (one cluster-reduced launch: U fp32, sU bf16)
 //                       -> fused dequant GEMM (CTA pairs for large M) with the
 //                       LoRA term as extra K stages                       2 launches
@@ -319,34 +320,56 @@ qlora_status linear_backward(const qlora_nf4& W, const LevelTable& t, const void
       QLORA_TRY(rank_down(xl, A, m, K, span, ru, s));
       U = u;
     }
-    if (dX && gemv) {
-      // dX = dY W + s V A: CTA partials of the dequant GEMV, summed in order
-      float* fpart = reinterpret_cast<float*>(ws + L.fused_b);
-      int parts = 0;
-      QLORA_TRY(gemv_dgrad(w, t, dY, M, v, A, r, sc_dx, fpart, &parts, s));
-      ReduceArgs rx = reduce_args(fpart, parts, M, static_cast<int>(K),
-                                  static_cast<int>(K));
-      rx.o2 = dX;
-      rx.ld2 = K;
-      rx.a2 = 1.0f;
-      QLORA_TRY(splitk_reduce(rx, s));
-    } else if (dX) {
-      const FusedShape f = fused_shape(M, K, ceil_div(N, 64));
-      if (f.splits == 1) {
-        QLORA_TRY(tc_fused_dgrad(w, t, dY, M, sv, A, r, dX, f, st, s));
-      } else {
+    // dB and dA on the side stream, dX on the caller's (as for large M): they
+    // share only inputs, all ready once V (and U) are
+    SideStream* ss = nullptr;
+    QLORA_TRY(side_stream(&ss));
+    const cudaStream_t s2 = ss->stream;
+    if (cudaEventRecord(ss->fork, s) != cudaSuccess ||
+        cudaStreamWaitEvent(s2, ss->fork, 0) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+    auto main_work = [&]() -> qlora_status {
+      if (dX && gemv) {
+        // dX = dY W + s V A: CTA partials of the dequant GEMV, summed in order
         float* fpart = reinterpret_cast<float*>(ws + L.fused_b);
-        QLORA_TRY(tc_fused_dgrad(w, t, dY, M, sv, A, r, fpart, f, st, s));
-        ReduceArgs rx = reduce_args(fpart, f.splits, M, static_cast<int>(K), static_cast<int>(K));
+        int parts = 0;
+        QLORA_TRY(gemv_dgrad(w, t, dY, M, v, A, r, sc_dx, fpart, &parts, s));
+        ReduceArgs rx = reduce_args(fpart, parts, M, static_cast<int>(K),
+                                    static_cast<int>(K));
         rx.o2 = dX;
         rx.ld2 = K;
         rx.a2 = 1.0f;
         QLORA_TRY(splitk_reduce(rx, s));
+      } else if (dX) {
+        const FusedShape f = fused_shape(M, K, ceil_div(N, 64));
+        if (f.splits == 1) {
+          QLORA_TRY(tc_fused_dgrad(w, t, dY, M, sv, A, r, dX, f, st, s));
+        } else {
+          float* fpart = reinterpret_cast<float*>(ws + L.fused_b);
+          QLORA_TRY(tc_fused_dgrad(w, t, dY, M, sv, A, r, fpart, f, st, s));
+          ReduceArgs rx = reduce_args(fpart, f.splits, M, static_cast<int>(K), static_cast<int>(K));
+          rx.o2 = dX;
+          rx.ld2 = K;
+          rx.a2 = 1.0f;
+          QLORA_TRY(splitk_reduce(rx, s));
+        }
       }
-    }
-    if (dX && o.mask) QLORA_TRY(dropout_dx(dX, v, r, A, o.mask, M, K, r, sc * o.keep, s));
-    QLORA_TRY(small_grad_b(dY, U, m, N, r, sc, accumulate, dB, s));
-    return small_grad_a(v, xl, m, K, r, sc * o.keep, accumulate, dA, s);
+      if (dX && o.mask) QLORA_TRY(dropout_dx(dX, v, r, A, o.mask, M, K, r, sc * o.keep, s));
+      return QLORA_OK;
+    };
+    auto side_work = [&]() -> qlora_status {
+      QLORA_TRY(small_grad_b(dY, U, m, N, r, sc, accumulate, dB, s2));
+      return small_grad_a(v, xl, m, K, r, sc * o.keep, accumulate, dA, s2);
+    };
+    // the dX kernel is enqueued first so that it takes the SMs
+    const qlora_status st_main = main_work();
+    const qlora_status st_side = side_work();
+    // join on every path, so that nothing of this call runs past it on the side stream
+    const bool joined = cudaEventRecord(ss->join, s2) == cudaSuccess &&
+                        cudaStreamWaitEvent(s, ss->join, 0) == cudaSuccess;
+    if (st_side != QLORA_OK) return st_side;
+    if (st_main != QLORA_OK) return st_main;
+    return joined ? QLORA_OK : QLORA_ERR_CUDA;
   }
   if (use_tc(M, N, K, r)) {
     const TcLayout L = tc_layout(M, N, K, r);
