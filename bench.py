@@ -603,23 +603,24 @@ def time_single(name, steps, warmup, peaks, dev):
         end.record()
         torch.cuda.synchronize()
     del graph
-    # the fused kernels' times from a second graph of the same steps, with the
-    # library's launch events captured into it
-    kinds = (Q.QLORA_KERNEL_FUSED_FWD, Q.QLORA_KERNEL_FUSED_DGRAD)
-    Q.qlora_timing_begin(kinds, max_launches=4 * len(shapes) * steps + 16)
+    # the fused kernels' and the quantiser's times from a second graph of the
+    # same steps, with the library's launch events captured into it (an event
+    # before a fused kernel makes it start after its U or V launch ends, where
+    # the timed graph lets the two overlap)
+    kinds = (Q.QLORA_KERNEL_FUSED_FWD, Q.QLORA_KERNEL_FUSED_DGRAD, Q.QLORA_KERNEL_QUANTIZE)
+    Q.qlora_timing_begin(kinds, max_launches=6 * len(shapes) * steps + 16)
     graph = capture()
     graph.replay()
     torch.cuda.synchronize()
     del graph  # it refers to the library's timing events
     kt = Q.qlora_timing_end()
-    Q.qlora_timing_begin((Q.QLORA_KERNEL_QUANTIZE, Q.QLORA_KERNEL_LORA_GEMM),
-                         max_launches=8 * len(shapes) * steps + 16)
+    # the rank-r products from eager launches of the same steps
+    Q.qlora_timing_begin((Q.QLORA_KERNEL_LORA_GEMM,), max_launches=8 * len(shapes) * steps + 16)
     for i in range(steps):
         step(sets[i % n_sets])
     torch.cuda.synchronize()
     kt2 = Q.qlora_timing_end()
-    for k in (Q.QLORA_KERNEL_QUANTIZE, Q.QLORA_KERNEL_LORA_GEMM):
-        kt[k] = kt2[k]
+    kt[Q.QLORA_KERNEL_LORA_GEMM] = kt2[Q.QLORA_KERNEL_LORA_GEMM]
     for g in sets:
         for s in g:
             Q.qlora_check(s.fws)
