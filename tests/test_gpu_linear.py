@@ -101,6 +101,19 @@ def test_attention_projection_4096(attn):
     assert torch.equal(dA, dA2) and torch.equal(dB, dB2)
 
 
+@pytest.mark.parametrize("M", [5120, 7168])
+def test_rank_splits_that_do_not_divide_the_row_tile(attn, M):
+    """5120 and 7168 tokens split the contraction of U = X A^T and V = dY B
+    7 and 5 ways when the clusters are resident (fewer otherwise): the
+    cluster's reduce then gives its last CTA a shorter slice of the 128 rows."""
+    shape, inp0, w_hat = attn
+    inp = WL.linear_inputs(shape, M, 0)
+    assert torch.equal(inp["W"], inp0["W"])  # the same W, so the same oracle weight
+    rows = np.sort(np.random.default_rng(M).choice(M, 64, replace=False))
+    rows = np.concatenate([[0], rows, [M - 1]])
+    _run(inp, shape.alpha, rows=rows, w_hat=w_hat)
+
+
 @pytest.fixture(scope="module", params=[0, 1], ids=["gate_up", "down"])
 def mlp(request):
     shape = WL.WORKLOADS["mlp_11008"].linears[request.param]
