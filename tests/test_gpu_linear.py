@@ -74,6 +74,9 @@ def test_single_linear_256():
     (4000, 2600, 640, 16), (4000, 640, 2624, 16),
     # two tokens (dequant GEMVs): K below one 1024-column group, and a ragged second group
     (2, 200, 320, 16), (2, 4104, 1088, 24),
+    # ranks that need more LoRA stages than the pipeline has slots: CTA pairs,
+    # decode sizes, and a rank that is not a multiple of 64
+    (600, 512, 1024, 256), (520, 384, 704, 200), (1, 1024, 1024, 256), (16, 520, 2048, 136),
 ])
 def test_ragged_shapes(M, N, K, r):
     inp, alpha = _inputs(N, K, r, M, 1000 + M, b_std=0.05)
