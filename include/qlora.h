@@ -224,7 +224,7 @@ qlora_status qlora_linear_bwd_multi(const qlora_nf4* W, const void* A, const voi
  * result can be quantised again with qlora_quantize.  For r a multiple of 8 the
  * rank-r product runs on the tensor cores; its device-side waits are bounded,
  * and as the call takes no status word, a wait that gives up (it does not in
- * correct operation) leaves NaN in its 128 x 256 tile of W_out. */
+ * correct operation) leaves NaN in its 128 x 128 tile of W_out. */
 qlora_status qlora_merge(const qlora_nf4* W, const void* A, const void* B, int32_t r,
                          float alpha, void* W_out, void* stream);
 
